@@ -1,0 +1,353 @@
+"""Benchmark of the exact attention forward on B200.
+
+Default workload: the dense MHA prefill (B=2, Hq=Hkv=32, N=8192, d=128, causal,
+5% of key rows x4), bf16 inputs resident in HBM.  One step = one forward over
+the whole batch (one kernel launch).  Metric: TFLOP/s counting 4*d FLOPs per
+visible (query, key) pair.  Inputs (384 MiB of q, k, v) are larger than the
+126 MB L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload dense|gqa|swa|long|tiny] [--no-cpu-baseline]
+
+With --gpus N > 1 the script runs under torchrun, one rank per GPU; every rank
+runs its own shard of the global batch (weak scaling, no data-path collective)
+and rank 0 prints one JSON line with the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from harness.inputs import WORKLOADS, make_qkv, sample_rows  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s (bf16, causal/window-adjusted) and % of B200 dense peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["exact_io_aware_72_b200/csrc/attn_fwd.cu", "exact_io_aware_72_b200/csrc/attn_fwd_kernel.cuh",
+                  "exact_io_aware_72_b200/csrc/sm100_ptx.cuh"]
+# DRAM bytes per launch of the forward kernel from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the kernel
+# sources it was taken on; reported only while the sources still match.
+NCU_TRAFFIC = {}
+
+
+def visible_pairs(N: int, mask: str, window) -> int:
+    """Visible (query, key) pairs of one head: N^2, N(N+1)/2, or N w - w(w-1)/2."""
+    if mask == "full":
+        return N * N
+    if mask == "causal" or (mask == "sliding_window" and window >= N):
+        return N * (N + 1) // 2
+    w = window
+    return N * w - w * (w - 1) // 2
+
+
+def workload_flops(w, batch: int) -> int:
+    return 4 * batch * w.Hq * w.d * visible_pairs(w.N, w.mask, w.window)
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while it runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.marks = [None, None]
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu=timestamp,{self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, i):
+        self.marks[i] = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        t0, t1 = self.marks
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if t0 is not None and not (t0 - 0.05 <= ts <= t1 + 0.15):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (a timing reduction, not data)."""
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------- oracle (CPU)
+def oracle_sample(w, q, k, v, rows, heads, scale):
+    """Time the fp64 oracle on `rows` of `heads` (list of (b, h)); returns
+    (seconds, visible-pair FLOPs done, threads)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    g = w.Hq // w.Hkv
+    # host copies prepared outside the timed region
+    work = []
+    for b, h in heads:
+        work.append((q[b:b + 1, h:h + 1].float().cpu().numpy(), k[b:b + 1, h // g:h // g + 1].float().cpu().numpy(),
+                     v[b:b + 1, h // g:h // g + 1].float().cpu().numpy()))
+    t0 = time.perf_counter()
+    for qh, kh, vh in work:
+        oracle.attention(qh, kh, vh, scale, w.mask_kind, w.window, rows=rows)
+    dt = time.perf_counter() - t0
+    counts = oracle.visible_count_per_row(w.N, w.mask_kind, w.window)[rows]
+    flops = 4 * w.d * int(counts.sum()) * len(heads)
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return dt, flops, threads
+
+
+def cpu_baseline(w, q, k, v, target_s=15.0):
+    """Oracle on host cores on a bounded sample of the workload (about target_s
+    seconds): seeded query rows of as many heads as fit, all heads if they fit."""
+    rows = sample_rows(w.N, w.window, w.seed + 100, count=min(w.N, 256))
+    dt, _, _ = oracle_sample(w, q, k, v, rows, [(0, 0)], w.scale)
+    n_heads = max(1, min(w.B * w.Hq, int(target_s / max(dt, 1e-3))))
+    if n_heads == w.B * w.Hq and dt * n_heads < target_s / 2 and len(rows) < w.N:
+        rows = sample_rows(w.N, w.window, w.seed + 100,
+                           count=min(w.N, int(len(rows) * target_s / max(dt * n_heads, 1e-3) / 2)))
+    heads = [(i // w.Hq, i % w.Hq) for i in range(n_heads)]
+    dt, flops, threads = oracle_sample(w, q, k, v, rows, heads, w.scale)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{len(rows)} seeded query rows x {n_heads} heads of the {w.name} workload "
+                      f"(fp64 NumPy, scores materialised), {dt:.1f} s",
+            "seconds": dt}
+
+
+# ----------------------------------------------------------------- arms
+def run_reference(args, w):
+    """The oracle as the reference arm: each step is a bounded sample of the
+    workload (64 seeded rows of a few heads) on the host cores."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, device="cpu", sharp=w.sharp)
+    rows = sample_rows(w.N, w.window, w.seed + 100, count=64)
+    heads = [(0, h) for h in range(min(4, w.Hq))]
+    for _ in range(args.warmup):
+        oracle_sample(w, q, k, v, rows, heads[:1], w.scale)
+    total_s, total_f, threads = 0.0, 0, 1
+    for _ in range(args.steps):
+        dt, fl, threads = oracle_sample(w, q, k, v, rows, heads, w.scale)
+        total_s += dt
+        total_f += fl
+    value = total_f / total_s / 1e12
+    sample = f"{len(rows)} seeded query rows x {len(heads)} heads of the {w.name} workload per step (fp64 NumPy)"
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000 * total_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                       "mask": w.mask, "window": w.window, "global_batch": w.B, "seq_len": w.N,
+                       "parallelism": "cpu"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w):
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    from exact_io_aware_72_b200 import fwd, fwd_host
+
+    # Each rank runs its own shard of the global batch: B sequences seeded by rank.
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed + 1000 * rank, device=device, sharp=w.sharp)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    flops = workload_flops(w, w.B)
+
+    def step():
+        fwd(q, k, v, scale=w.scale, mask=w.mask, window=w.window, out=out, lse=lse, stream=stream)
+
+    clocks = ClockSampler(local)
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    clocks.mark(0)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    evs[0].record(stream)
+    for i in range(args.steps):
+        step()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize(device)
+    clocks.mark(1)
+    barrier(world, device)
+    per_launch_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    total_ms = evs[0].elapsed_time(evs[-1])
+    total_ms = max_over_ranks(total_ms, world, device)
+    clk = clocks.stop() if rank == 0 else None
+
+    # End to end through the public host-buffer call: pinned q, k, v in, out and lse back.
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    for _ in range(2):
+        fwd_host(hq, hk, hv, device=device, scale=w.scale, mask=w.mask, window=w.window)
+    e2e_steps = max(3, min(args.steps, 20))
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        fwd_host(hq, hk, hv, device=device, scale=w.scale, mask=w.mask, window=w.window)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        avg_launch_s = statistics.mean(per_launch_ms) / 1e3
+        achieved = flops / avg_launch_s / 1e12
+        peak = float(peaks["bf16_tflops"])
+        value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+        traffic = NCU_TRAFFIC.get((w.name, kernel_hash()))
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                       "mask": w.mask, "window": w.window, "sharp_rows": w.sharp,
+                       "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "frac_of_peak": value / world / peak,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak))},
+            "gpu_launches": args.steps,
+            "clocks": clk,
+            "e2e": {"value": world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, q, k, v, target_s=args.cpu_seconds)
+            line["cpu_baseline"].pop("seconds", None)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="dense")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,144 @@
+"""Python binding of the C ABI in include/attn.h (argument marshalling only).
+
+Every step of the forward runs in the sm_100a kernels of ``libattn_b200.so``;
+PyTorch only provides device memory and the current stream.  There is no
+fallback: if the library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+MASKS = {"full": 0, "causal": 1, "sliding_window": 2}
+STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_MISALIGNED",
+          4: "ATTN_ERR_CUDA", 5: "ATTN_ERR_TIMEOUT"}
+ATTN_ERR_TIMEOUT = 5
+LIB_NAME = "libattn_b200.so"
+EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_status_string", "attn_debug_error", "attn_fwd_num_work_items")
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class FwdOptions(ctypes.Structure):
+    _fields_ = [("wait_timeout_ns", ctypes.c_uint64), ("inject_stall", ctypes.c_int),
+                ("grid_ctas", ctypes.c_int)]
+
+
+def lib_path() -> str:
+    return os.path.join(os.path.dirname(os.path.abspath(__file__)), LIB_NAME)
+
+
+def load_library():
+    """Load libattn_b200.so (built in-tree); raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = lib_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{LIB_NAME} is not built; run `python -m exact_io_aware_72_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    fwd_args = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, ctypes.c_float, ctypes.c_int, i64, vp]
+    lib.attn_fwd.argtypes = fwd_args
+    lib.attn_fwd.restype = ctypes.c_int
+    lib.attn_fwd_ex.argtypes = fwd_args + [ctypes.POINTER(FwdOptions)]
+    lib.attn_fwd_ex.restype = ctypes.c_int
+    lib.attn_status_string.argtypes = [ctypes.c_int]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    lib.attn_debug_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    lib.attn_debug_error.restype = ctypes.c_int
+    lib.attn_fwd_num_work_items.argtypes = [i64, i64, i64, i64, i64, ctypes.c_int, i64]
+    lib.attn_fwd_num_work_items.restype = i64
+    _lib = lib
+    return lib
+
+
+def _check(t: torch.Tensor, name: str, dtype, ndim):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype or t.dim() != ndim or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor with {ndim} dims")
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
+        mask: str = "causal", window: Optional[int] = None, out: Optional[torch.Tensor] = None,
+        lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+        wait_timeout_ns: int = 0, inject_stall: bool = False, grid_ctas: int = 0
+        ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Exact attention forward: returns (out bf16 [B,Hq,N,d], lse fp32 [B,Hq,N]).
+
+    q: [B,Hq,N,d], k/v: [B,Hkv,N,d], bf16, contiguous, on one CUDA device.
+    ``mask`` is "full", "causal" or "sliding_window" (keys i-window < j <= i).
+    The launch is asynchronous on ``stream`` (default: the current stream).
+    """
+    lib = load_library()
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k, "k", torch.bfloat16, 4)
+    _check(v, "v", torch.bfloat16, 4)
+    B, Hq, N, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if (Bk, Nk, dk) != (B, N, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("q, k, v shapes disagree")
+    if mask not in MASKS:
+        raise ValueError(f"mask must be one of {sorted(MASKS)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    opts = FwdOptions(int(wait_timeout_ns), 1 if inject_stall else 0, int(grid_ctas))
+    with torch.cuda.device(q.device):
+        st = lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                             B, Hq, Hkv, N, d, float(scale), MASKS[mask],
+                             int(window) if window is not None else 0, ctypes.c_void_p(stream.cuda_stream),
+                             ctypes.byref(opts))
+    if st != 0:
+        raise AttnError(st, "attn_fwd")
+    return out, lse
+
+
+def debug_error(stream: Optional[torch.cuda.Stream] = None, device=None) -> Tuple[int, int]:
+    """Synchronise and read/clear the device error word: (status, raw code)."""
+    lib = load_library()
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    code = ctypes.c_int(0)
+    with torch.cuda.device(stream.device):
+        st = lib.attn_debug_error(ctypes.c_void_p(stream.cuda_stream), ctypes.byref(code))
+    return st, code.value
+
+
+def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, device="cuda", **kw):
+    """End-to-end call on HOST tensors (ideally pinned): copies q, k, v to the
+    device, runs the forward, and copies out and lse back to host memory."""
+    dq = q.to(device, non_blocking=True)
+    dk = k.to(device, non_blocking=True)
+    dv = v.to(device, non_blocking=True)
+    out, lse = fwd(dq, dk, dv, **kw)
+    pin = q.is_pinned()
+    ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=pin)
+    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=pin)
+    ho.copy_(out, non_blocking=True)
+    hl.copy_(lse, non_blocking=True)
+    torch.cuda.current_stream(dq.device).synchronize()
+    return ho, hl
+
+
+def num_work_items(B, Hq, Hkv, N, d, mask="causal", window=None) -> int:
+    return int(load_library().attn_fwd_num_work_items(B, Hq, Hkv, N, d, MASKS[mask],
+                                                      int(window) if window is not None else 0))

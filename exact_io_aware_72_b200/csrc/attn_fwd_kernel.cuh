@@ -1,0 +1,646 @@
+// Exact attention forward for sm_100a: one persistent, warp-specialised kernel.
+//
+// What it computes is masked softmax attention with an online softmax
+// ("Efficient attention: long context and sub-quadratic variants",
+// stanleyjacob.dev, sections "Implementation, twice" and "FlashAttention: exact
+// attention, IO-aware"): scores are formed tile by tile on chip, folded into a
+// running (max, sum) per query row, and the N x N matrix never reaches HBM.
+//
+// CTA organisation (384 threads = 3 warpgroups, one CTA per SM, persistent):
+//   warps 0-3   softmax for query tile 0 (thread = one query row = one TMEM lane)
+//   warps 4-7   softmax for query tile 1
+//   warp  8     TMA loader: Q tiles once per work item, K/V tiles through a ring
+//   warps 9-10  tcgen05 issuers, one thread per query tile: S = Q K^T and
+//               O += P V; warp 9 also owns the TMEM allocation
+//   warp  11    idle
+// Registers: launched at 168 per thread; the softmax warpgroups raise theirs to
+// 208 and the third warpgroup drops to 88 (2*128*208 + 128*88 = 384*168).
+// A work item is two 128-row query tiles that read the same K/V tiles: two query
+// heads of one KV group (GQA with an even group size) or two consecutive query
+// blocks of one head.  The two tiles ping-pong: while the softmax warps of one
+// tile work, the tensor core runs the other tile's matmuls.
+//
+// TMEM (512 columns x 128 lanes, fp32): S0 [0,128) S1 [128,256) O0 and O1 after
+// them.  P (bf16, two per column) overwrites the first 64 columns of its S tile.
+//
+// Every mbarrier wait is bounded by a global-timer limit; a wait that gives up
+// records a code in the device error word and raises a CTA-wide abort flag, and
+// all roles then leave their loops, drain what they issued, and free TMEM.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace attn_sm100 {
+
+constexpr int kBlockM = 128;    // query rows per tile
+constexpr int kBlockN = 128;    // keys per K/V tile
+constexpr int kThreads = 384;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSoftmaxRegs = 208;
+constexpr uint32_t kOtherRegs = 88;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * 168, "register split exceeds launch");
+constexpr float kLn2 = 0.6931471805599453f;
+// The running max is only moved when a row's max grows by more than this many
+// powers of two; until then P may exceed 1 by up to 2^8, which fp32 sums and
+// bf16 P carry without loss.  The final O / l uses the same max, so the result
+// is unchanged.
+constexpr float kRescaleThreshold = 8.0f;
+
+enum : int { kMaskFull = 0, kMaskCausal = 1, kMaskWindow = 2 };
+
+// Error codes: role in bits 8..11, barrier index in bits 0..7.
+enum : int { kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3 };
+
+struct FwdParams {
+  CUtensorMap tm_q;  // [B*Hq, N, d] bf16, box 64 x 128, 128B swizzle
+  CUtensorMap tm_k;  // [B*Hkv, N, d]
+  CUtensorMap tm_v;  // [B*Hkv, N, d]
+  __nv_bfloat16* out;
+  float* lse;
+  int* err;          // device error word
+  int B, Hq, Hkv, N;
+  int group;         // Hq / Hkv
+  int mask_kind;
+  int window;
+  float scale_log2;  // scale * log2(e)
+  int pair_heads;    // 1: the two tiles are two heads of one KV group
+  int num_mblk;      // ceil(N / 128)
+  int row_units;     // query-block units per head (unit = block or block pair)
+  int head_units;    // items per row unit
+  int num_items;
+  unsigned long long timeout_ns;
+  int inject_stall;
+};
+
+template <int D>
+struct SmemLayout {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int kChunks = D / 64;                         // 128-byte column chunks
+  static constexpr uint32_t kChunkBytes = kBlockM * 128;         // 128 rows x 128 B
+  static constexpr uint32_t kTileBytes = kChunks * kChunkBytes;  // one Q, K or V tile
+  static constexpr int kStages = (D == 128) ? 5 : 8;             // K/V ring slots
+  static constexpr uint32_t kQOff = 0;
+  static constexpr uint32_t kKVOff = 2 * kTileBytes;
+  static constexpr uint32_t kBarOff = kKVOff + kStages * kTileBytes;
+  static constexpr int kQFull = 0;
+  static constexpr int kQEmpty = 1;
+  static constexpr int kKVFull = 2;
+  static constexpr int kKVEmpty = kKVFull + kStages;
+  static constexpr int kSFull = kKVEmpty + kStages;
+  static constexpr int kPFull = kSFull + 2;
+  static constexpr int kODone = kPFull + 2;
+  static constexpr int kOFree = kODone + 2;
+  static constexpr int kFin = kOFree + 2;
+  static constexpr int kTurn = kFin + 2;
+  static constexpr int kNumBars = kTurn + 2;
+  static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr uint32_t kBytes = kMiscOff + 16;
+  static constexpr uint32_t kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
+  static constexpr uint32_t kSCol0 = 0, kSCol1 = 128;
+  static constexpr uint32_t kOCol0 = 256, kOCol1 = 256 + D;
+};
+
+// ------------------------------------------------------------ work items
+struct WorkItem {
+  int b, hkv;
+  int head[2];
+  int mblk[2];
+  int valid[2];
+  int lo[2], hi[2];  // KV tile range of each query tile
+  int lo_u, hi_u;    // union of the two ranges
+};
+
+__device__ __forceinline__ void kv_range(const FwdParams& p, int m, int& lo, int& hi) {
+  const int r0 = m * kBlockM;
+  const int r1 = min(r0 + kBlockM - 1, p.N - 1);
+  if (p.mask_kind == kMaskFull) {
+    lo = 0;
+    hi = p.num_mblk - 1;
+  } else {
+    hi = r1 / kBlockN;
+    lo = (p.mask_kind == kMaskWindow) ? max(0, r0 - p.window + 1) / kBlockN : 0;
+  }
+}
+
+// Items are ordered longest first (row unit descending), heads inside.
+__device__ __forceinline__ WorkItem decode_item(const FwdParams& p, int idx) {
+  WorkItem it;
+  const int r = p.row_units - 1 - idx / p.head_units;
+  const int u = idx % p.head_units;
+  if (p.pair_heads) {
+    const int hpairs = p.Hq >> 1;
+    it.b = u / hpairs;
+    const int hp = u - it.b * hpairs;
+    it.head[0] = 2 * hp;
+    it.head[1] = 2 * hp + 1;
+    it.mblk[0] = it.mblk[1] = r;
+  } else {
+    it.b = u / p.Hq;
+    it.head[0] = it.head[1] = u - it.b * p.Hq;
+    it.mblk[0] = 2 * r;
+    it.mblk[1] = 2 * r + 1;
+  }
+  it.hkv = it.head[0] / p.group;
+  it.lo_u = 0x7fffffff;
+  it.hi_u = -1;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    it.valid[t] = it.mblk[t] < p.num_mblk;
+    if (it.valid[t]) {
+      kv_range(p, it.mblk[t], it.lo[t], it.hi[t]);
+      it.lo_u = min(it.lo_u, it.lo[t]);
+      it.hi_u = max(it.hi_u, it.hi[t]);
+    } else {
+      it.lo[t] = 1;
+      it.hi[t] = 0;
+    }
+  }
+  return it;
+}
+
+// Does KV tile j need element-wise masking for query block m?
+__device__ __forceinline__ bool tile_is_partial(const FwdParams& p, int m, int j) {
+  const int r0 = m * kBlockM, c0 = j * kBlockN;
+  bool partial = (c0 + kBlockN > p.N);
+  if (p.mask_kind != kMaskFull) partial |= (c0 + kBlockN - 1 > r0);
+  if (p.mask_kind == kMaskWindow) partial |= (c0 <= r0 + kBlockM - 1 - p.window);
+  return partial;
+}
+
+// Static persistent schedule: round k hands item k*G + c (even k) or
+// k*G + G-1-c (odd k) to CTA c, pairing heavy items with light ones.
+struct Schedule {
+  int k, cta, grid, total;
+  __device__ Schedule(int cta_, int grid_, int total_) : k(0), cta(cta_), grid(grid_), total(total_) {}
+  __device__ __forceinline__ bool next(int& idx) {
+    while (true) {
+      const int base = k * grid;
+      if (base >= total) return false;
+      idx = base + ((k & 1) ? (grid - 1 - cta) : cta);
+      ++k;
+      if (idx < total) return true;
+    }
+  }
+};
+
+// ------------------------------------------------------------ bounded waits
+struct Waiter {
+  uint64_t limit_ns;
+  volatile int* abort_flag;
+  int* err;
+  // Wait for the phase of `bar` with parity `parity`; false if the CTA aborts.
+  __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, int code) const {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        atomicCAS(err, 0, code);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+  // Wait for work this thread itself started (copies, MMAs) to finish, even
+  // after an abort; still bounded by the time limit.
+  __device__ __forceinline__ bool drain(uint32_t bar, uint32_t parity, int code) const {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+      if (global_timer_ns() - t0 > limit_ns) {
+        atomicCAS(err, 0, code);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+    return true;
+  }
+};
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// ------------------------------------------------------------ roles
+template <int D>
+__device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sbase, const Waiter& w) {
+  using L = SmemLayout<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  const uint64_t pol_kv = l2_policy_evict_last();
+  const uint64_t pol_q = l2_policy_evict_first();
+  tma_prefetch_map(&p.tm_q);
+  tma_prefetch_map(&p.tm_k);
+  tma_prefetch_map(&p.tm_v);
+
+  uint32_t kv_n = 0;  // K/V loads issued so far
+  uint32_t q_issued = 0;
+  int items = 0;
+  bool ok = !p.inject_stall;
+  Schedule sched(blockIdx.x, gridDim.x, p.num_items);
+  int idx;
+  while (ok && sched.next(idx)) {
+    const WorkItem it = decode_item(p, idx);
+    if (items > 0 && !w.wait(bar(L::kQEmpty), (items - 1) & 1, (kRoleProducer << 8) | L::kQEmpty)) {
+      ok = false;
+      break;
+    }
+    const uint32_t qbytes = (it.valid[0] + it.valid[1]) * L::kTileBytes;
+    mbar_arrive_expect_tx(bar(L::kQFull), qbytes);
+    ++q_issued;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if (!it.valid[t]) continue;
+#pragma unroll
+      for (int c = 0; c < L::kChunks; ++c)
+        tma_load_3d(sbase + L::kQOff + t * L::kTileBytes + c * L::kChunkBytes, &p.tm_q, bar(L::kQFull),
+                    c * 64, it.mblk[t] * kBlockM, it.b * p.Hq + it.head[t], pol_q);
+    }
+    for (int j = it.lo_u; j <= it.hi_u && ok; ++j) {
+#pragma unroll
+      for (int kv = 0; kv < 2; ++kv) {
+        const uint32_t slot = kv_n % L::kStages;
+        if (kv_n >= (uint32_t)L::kStages &&
+            !w.wait(bar(L::kKVEmpty + slot), ((kv_n / L::kStages) - 1) & 1,
+                    (kRoleProducer << 8) | (L::kKVEmpty + slot))) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(L::kKVFull + slot), L::kTileBytes);
+        const CUtensorMap* map = kv ? &p.tm_v : &p.tm_k;
+#pragma unroll
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(sbase + L::kKVOff + slot * L::kTileBytes + c * L::kChunkBytes, map,
+                      bar(L::kKVFull + slot), c * 64, j * kBlockN, it.b * p.Hkv + it.hkv, pol_kv);
+        ++kv_n;
+      }
+    }
+    ++items;
+  }
+  // Drain: every copy this thread started must land before the CTA exits.
+  for (uint32_t s = 0; s < (uint32_t)L::kStages; ++s) {
+    if (kv_n > s) {
+      const uint32_t last = s + ((kv_n - 1 - s) / L::kStages) * L::kStages;  // last load into slot s
+      w.drain(bar(L::kKVFull + s), (last / L::kStages) & 1, (kRoleProducer << 8) | (L::kKVFull + s));
+    }
+  }
+  if (q_issued > 0) w.drain(bar(L::kQFull), (q_issued - 1) & 1, (kRoleProducer << 8) | L::kQFull);
+}
+
+// One issuing thread per query tile t.  For each KV tile j of the item:
+//   O_t += P_t(j-1) V_{j-1}   (once the softmax has written P_t(j-1))
+//   S_t  = Q_t K_j^T          (after that P V in issue order, since P aliases S)
+// and releases K_j / V_{j-1} / Q with commits; the other tile's thread does the
+// same, so each ring slot is freed after both threads' reads complete.
+template <int D>
+__device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tmem, const Waiter& w,
+                                         int t) {
+  using L = SmemLayout<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false);
+  constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, true);
+  const uint32_t s_tmem = tmem + (t ? L::kSCol1 : L::kSCol0);
+  const uint32_t o_tmem = tmem + (t ? L::kOCol1 : L::kOCol0);
+  // Descriptor bases: Q_t (K-major), ring slot 0 as K (K-major) and as V
+  // (MN-major, d chunks 16 KB apart).  Per-MMA offsets are added to the start
+  // address field (16-byte units).
+  const uint64_t q_desc = smem_desc_sw128(sbase + L::kQOff + t * L::kTileBytes, 16, 1024);
+  const uint64_t k_desc0 = smem_desc_sw128(sbase + L::kKVOff, 16, 1024);
+  const uint64_t v_desc0 = smem_desc_sw128(sbase + L::kKVOff, L::kChunkBytes, 1024);
+  const int code = (kRoleMma << 8) | (t << 7);
+
+  uint32_t kv_n = 0;
+  uint32_t p_cnt = 0;
+  int items = 0;
+  bool ok = true;
+  Schedule sched(blockIdx.x, gridDim.x, p.num_items);
+  int idx;
+  while (ok && sched.next(idx)) {
+    const WorkItem it = decode_item(p, idx);
+    const int valid = t ? it.valid[1] : it.valid[0];
+    const int lo = t ? it.lo[1] : it.lo[0];
+    const int hi = t ? it.hi[1] : it.hi[0];
+    if (!w.wait(bar(L::kQFull), items & 1, code | L::kQFull)) break;
+    tc_fence_after_sync();
+    bool pend = false;
+    bool first_pv = true;
+
+    // O_t += P_t V for the V tile with load index vn.
+    auto issue_pv = [&](uint32_t vn) -> bool {
+      if (first_pv && items > 0 && !w.wait(bar(L::kOFree + t), (items - 1) & 1, code | (L::kOFree + t)))
+        return false;
+      if (!w.wait(bar(L::kPFull + t), p_cnt & 1, code | (L::kPFull + t))) return false;
+      ++p_cnt;
+      const uint32_t vslot = vn % L::kStages;
+      if (!w.wait(bar(L::kKVFull + vslot), (vn / L::kStages) & 1, code | (L::kKVFull + vslot))) return false;
+      tc_fence_after_sync();
+      const uint64_t vd = v_desc0 + ((vslot * L::kTileBytes) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < kBlockN / 16; ++kk) {
+        // 16 keys = two 8-row swizzle atoms = 2048 B further into the V tile.
+        mma_bf16_ts(o_tmem, s_tmem + kk * 8, vd + ((kk * 2048) >> 4), idesc_o, (kk > 0 || !first_pv) ? 1u : 0u);
+      }
+      first_pv = false;
+      pend = false;
+      return true;
+    };
+
+    for (int j = it.lo_u; j <= it.hi_u; ++j) {
+      const uint32_t kslot = kv_n % L::kStages;
+      if (pend && !issue_pv(kv_n - 1)) {
+        ok = false;
+        break;
+      }
+      if (!w.wait(bar(L::kKVFull + kslot), (kv_n / L::kStages) & 1, code | (L::kKVFull + kslot))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      if (valid && j >= lo && j <= hi) {
+        const uint64_t kd = k_desc0 + ((kslot * L::kTileBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          // K-major operands: 16 elements = 32 B inside a 128 B swizzled row,
+          // the next 64 columns 16 KB further.
+          const uint32_t off = ((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(s_tmem, q_desc + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(L::kSFull + t));
+        pend = true;
+      }
+      tc_commit(bar(L::kKVEmpty + kslot));                                   // K_j read
+      if (j > it.lo_u) tc_commit(bar(L::kKVEmpty + (kv_n - 1) % L::kStages));  // V_{j-1} read
+      if (j == it.hi_u) tc_commit(bar(L::kQEmpty));                          // Q read
+      kv_n += 2;
+    }
+    if (!ok) break;
+    if (pend && !issue_pv(kv_n - 1)) break;
+    tc_commit(bar(L::kKVEmpty + (kv_n - 1) % L::kStages));  // V_hi read
+    if (first_pv && items > 0 && !w.wait(bar(L::kOFree + t), (items - 1) & 1, code | (L::kOFree + t))) break;
+    tc_commit(bar(L::kODone + t));
+    ++items;
+  }
+  // Drain: every MMA this thread issued must complete before TMEM is freed.
+  tc_commit(bar(L::kFin + t));
+  w.drain(bar(L::kFin + t), 0, code | (L::kFin + t));
+}
+
+template <int D>
+__device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tmem,
+                                             const Waiter& w, int warp, int lane) {
+  using L = SmemLayout<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  const int t = warp >> 2;
+  const int quarter = warp & 3;
+  const int row_in_tile = quarter * 32 + lane;
+  const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t tS = tmem + lane_bits + (t ? L::kSCol1 : L::kSCol0);
+  const uint32_t tO = tmem + lane_bits + (t ? L::kOCol1 : L::kOCol0);
+  const float c = p.scale_log2;
+
+  uint32_t s_cnt = 0;
+  uint32_t turn_cnt = 0;
+  int items = 0;
+  bool ok = true;
+  Schedule sched(blockIdx.x, gridDim.x, p.num_items);
+  int idx;
+  while (ok && sched.next(idx)) {
+    const WorkItem it = decode_item(p, idx);
+    // This warp's tile, picked with selects so the item stays in registers.
+    const int mblk = t ? it.mblk[1] : it.mblk[0];
+    const int head = t ? it.head[1] : it.head[0];
+    const int valid = t ? it.valid[1] : it.valid[0];
+    const int lo = t ? it.lo[1] : it.lo[0];
+    const int hi = t ? it.hi[1] : it.hi[0];
+    const int row = mblk * kBlockM + row_in_tile;
+    float m_run = -INFINITY;
+    float l_run = 0.f;   // sum of P as written (bf16), normalises O
+    float l_lse = 0.f;   // sum of P in fp32, for the log-sum-exp
+    // Both softmax warpgroups walk the item's whole KV range so they can hand
+    // the turn token back and forth: the exp loop of one tile runs while
+    // the tensor core works on the other tile (the exp unit is the shared
+    // bottleneck), whether or not a tile has work at a given step.
+    for (int j = it.lo_u; j <= it.hi_u; ++j) {
+      const bool active = valid && j >= lo && j <= hi;
+      float s[128];
+      if (active) {
+        bool got = w.wait(bar(L::kSFull + t), s_cnt & 1, (kRoleSoftmax << 8) | (L::kSFull + t));
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        ++s_cnt;
+        tc_fence_after_sync();
+        uint32_t sr[128];
+        tmem_load_128cols(tS, sr);
+#pragma unroll
+        for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
+        if (tile_is_partial(p, mblk, j)) {
+          const int c0 = j * kBlockN;
+          const int hi_i = ((p.mask_kind == kMaskFull) ? p.N - 1 : min(row, p.N - 1)) - c0;
+          const int lo_i = (p.mask_kind == kMaskWindow) ? row - p.window + 1 - c0 : -1;
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i > hi_i || i < lo_i) s[i] = -INFINITY;
+        }
+      }
+      bool need = false;
+      float alpha = 1.f;
+      float neg_base = 0.f;
+      if (active) {
+        // Row max: eight chains of three-input max (integer/ALU work, done
+        // before taking the turn so it overlaps the other tile's exp loop).
+        float mx[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mx[q] = s[q];
+#pragma unroll
+        for (int i = 8; i < 128; i += 2) mx[(i >> 1) & 7] = max3f(mx[(i >> 1) & 7], s[i], s[i + 1]);
+        const float tile_max = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+        const float m_new = fmaxf(m_run, tile_max * c);
+        need = m_new > m_run + kRescaleThreshold;
+        if (need) {
+          alpha = fast_exp2(m_run - m_new);
+          m_run = m_new;
+        }
+        neg_base = (m_run == -INFINITY) ? 0.f : -m_run;
+      }
+      {
+        bool got = w.wait(bar(L::kTurn + t), turn_cnt & 1, (kRoleSoftmax << 8) | (L::kTurn + t));
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        ++turn_cnt;
+      }
+      if (active) {
+        // p = 2^(s*c - m) on column pairs (packed fp32 FMA), then P to bf16 by
+        // rounding half up on the integer pipe (the fp32->bf16 convert would
+        // share the exp2 unit).  O is normalised by the sum of exactly these
+        // rounded values, so each row's weights stay a convex combination; the
+        // log-sum-exp uses the fp32 sum.  P goes to TMEM 16 columns at a time.
+        const uint64_t c2 = f32x2_pack(c, c);
+        const uint64_t nb2 = f32x2_pack(neg_base, neg_base);
+        uint64_t so2 = 0, sl2 = 0;  // (+0.f, +0.f)
+#pragma unroll
+        for (int chunk = 0; chunk < 4; ++chunk) {
+          if (chunk == 3) {
+            // Hand the turn over one chunk early: the other tile's wake-up
+            // overlaps the tail of this loop.
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::kTurn + (t ^ 1)));
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = chunk * 32 + 2 * i;
+            float x0, x1;
+            f32x2_unpack(f32x2_fma(f32x2_pack(s[e], s[e + 1]), c2, nb2), x0, x1);
+            const float p0 = fast_exp2(x0);
+            const float p1 = fast_exp2(x1);
+            const uint32_t u0 = __float_as_uint(p0) + 0x8000u;
+            const uint32_t u1 = __float_as_uint(p1) + 0x8000u;
+            pk[i] = __byte_perm(u0, u1, 0x7632);
+            so2 = f32x2_add(so2, f32x2_pack(__uint_as_float(u0 & 0xffff0000u), __uint_as_float(u1 & 0xffff0000u)));
+            sl2 = f32x2_add(sl2, f32x2_pack(p0, p1));
+          }
+          tmem_store_16cols(tS + chunk * 16, pk);
+        }
+        float so_lo, so_hi, sl_lo, sl_hi;
+        f32x2_unpack(so2, so_lo, so_hi);
+        f32x2_unpack(sl2, sl_lo, sl_hi);
+        l_run = l_run * alpha + (so_lo + so_hi);
+        l_lse = l_lse * alpha + (sl_lo + sl_hi);
+      }
+      if (!active) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::kTurn + (t ^ 1)));
+      } else {
+        if (j > lo && __any_sync(0xffffffffu, need)) {
+          // O of this row was last written by the P V of the previous tile; that
+          // MMA completed before this S tile did (in-order tcgen05 completion).
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_load_32cols(tO + cc * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_store_32cols(tO + cc * 32, o);
+          }
+        }
+        tmem_store_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::kPFull + t));
+      }
+    }
+    if (!ok) break;
+    // Epilogue: O / l to bf16, log-sum-exp to fp32.
+    bool got = w.wait(bar(L::kODone + t), items & 1, (kRoleSoftmax << 8) | (L::kODone + t));
+    if (!__all_sync(0xffffffffu, got)) break;
+    tc_fence_after_sync();
+    if (valid) {
+      const bool row_ok = row < p.N;
+      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      const size_t head_row = (static_cast<size_t>(it.b) * p.Hq + head) * p.N + (row_ok ? row : 0);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + head_row * D);
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_load_32cols(tO + cc * 32, o);
+        if (row_ok) {
+          uint32_t h[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            h[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[cc * 4 + v] = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+        }
+      }
+      if (row_ok) p.lse[head_row] = (m_run + __log2f(l_lse)) * kLn2;
+    }
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(L::kOFree + t));
+    ++items;
+  }
+  tmem_store_wait();
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
+  using L = SmemLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  if (threadIdx.x == 0) {
+    auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+    mbar_init(bar(L::kQFull), 1);
+    mbar_init(bar(L::kQEmpty), 2);             // one commit per MMA thread
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar(L::kKVFull + s), 1);
+      mbar_init(bar(L::kKVEmpty + s), 2);      // one commit per MMA thread
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(L::kSFull + t), 1);
+      mbar_init(bar(L::kPFull + t), 4);        // one arrival per softmax warp
+      mbar_init(bar(L::kODone + t), 1);
+      mbar_init(bar(L::kOFree + t), 4);        // one arrival per softmax warp
+      mbar_init(bar(L::kFin + t), 1);
+      mbar_init(bar(L::kTurn + t), 4);         // one arrival per warp of the other warpgroup
+    }
+    for (int i = 0; i < 4; ++i) mbar_arrive(bar(L::kTurn + 0));  // tile 0 starts with the turn
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const Waiter w{p.timeout_ns, abort_flag, p.err};
+
+  if (warp < 8) {
+    reg_alloc_raise<kSoftmaxRegs>();
+    softmax_role<D>(p, sbase, tmem, w, warp, lane);
+  } else {
+    reg_alloc_lower<kOtherRegs>();
+  }
+  if (warp == kProducerWarp) {
+    if (lane == 0) producer_role<D>(p, sbase, w);
+    __syncwarp();
+  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+    if (lane == 0) mma_role<D>(p, sbase, tmem, w, warp - kMmaWarp);
+    __syncwarp();
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace attn_sm100

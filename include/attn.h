@@ -1,0 +1,119 @@
+/*
+ * Exact attention forward for NVIDIA B200 (sm_100a): C ABI.
+ *
+ * Computes, for every batch b, query head h and query row i,
+ *
+ *     out[b,h,i,:] = sum_j softmax_j(scale * q[b,h,i,:] . k[b,g(h),j,:] + mask(i,j)) * v[b,g(h),j,:]
+ *     lse[b,h,i]   = ln sum_{j visible} exp(scale * q[b,h,i,:] . k[b,g(h),j,:])
+ *
+ * which is the masked softmax attention of "Efficient attention: long context and
+ * sub-quadratic variants" (stanleyjacob.dev), section "Implementation, twice"
+ * (masked_attention: masked scores are -inf before the softmax, each row is
+ * renormalised over its visible keys), computed tile by tile with an online
+ * softmax so the N x N score matrix never reaches HBM (same page, section
+ * "FlashAttention: exact attention, IO-aware").
+ *
+ * Masks (mask(i,j) = 0 where visible, -inf elsewhere):
+ *   ATTN_MASK_FULL            every key;
+ *   ATTN_MASK_CAUSAL          j <= i ("Efficient Attention: Flash Attention, Sliding
+ *                             Window, Sparse", creativeworksofknowledge.com, section "Code":
+ *                             is_causal=True);
+ *   ATTN_MASK_SLIDING_WINDOW  i - window < j <= i (stanleyjacob.dev, section
+ *                             "Sliding-window and local attention" and sliding_window_mask);
+ *                             a window >= N is exactly causal and is run as causal.
+ * Head sharing (GQA/MQA): query head h reads key/value head g(h) = h / (Hq / Hkv)
+ * ("Attention Mechanism Variants Beyond Self-Attention", tempatgunting.com, section
+ * "Multi-Query and Grouped-Query Attention": repeat_interleave on the head axis).
+ * The log-sum-exp output is not on those pages; it is the natural-log normaliser of
+ * each row's softmax, written so a caller can merge or recompute partial results.
+ */
+#ifndef ATTN_B200_ATTN_H_
+#define ATTN_B200_ATTN_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_MASK_FULL = 0,
+  ATTN_MASK_CAUSAL = 1,
+  ATTN_MASK_SLIDING_WINDOW = 2
+} attn_mask_kind;
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad mask, window < 1, scale not finite or <= 0,
+                                overlapping buffers */
+  ATTN_ERR_UNSUPPORTED = 2,  /* head dimension other than 64 or 128, or no sm_100 device */
+  ATTN_ERR_MISALIGNED = 3,   /* q, k, v or out not 16-byte aligned, lse not 4-byte aligned */
+  ATTN_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed (launch, tensor-map encode) */
+  ATTN_ERR_TIMEOUT = 5       /* a device-side wait gave up (reported by attn_debug_error) */
+} attn_status;
+
+/*
+ * attn_fwd: enqueue the forward on `stream` and return immediately.
+ *
+ *   q    device pointer, bf16, [B, Hq,  N, d], contiguous (d fastest), 16-byte aligned
+ *   k    device pointer, bf16, [B, Hkv, N, d], contiguous, 16-byte aligned
+ *   v    device pointer, bf16, [B, Hkv, N, d], contiguous, 16-byte aligned
+ *   out  device pointer, bf16, [B, Hq,  N, d], contiguous, 16-byte aligned; fully overwritten
+ *   lse  device pointer, fp32, [B, Hq,  N],    contiguous, 4-byte aligned; fully overwritten
+ *   B, Hq, Hkv, N >= 1; Hq % Hkv == 0; d in {64, 128}
+ *   scale      finite and > 0 (usually 1/sqrt(d)); multiplies q.k before the mask
+ *   mask_kind  an attn_mask_kind
+ *   window     >= 1 when mask_kind == ATTN_MASK_SLIDING_WINDOW, ignored otherwise
+ *   stream     CUDA stream (0 = legacy default stream) of the current device, which
+ *              must own all five buffers
+ *
+ * Ownership: the caller owns every buffer. The library allocates no device memory and
+ * never synchronises; out and lse are written by the kernel when the stream reaches it.
+ * out and lse must not overlap each other or the inputs (ATTN_ERR_INVALID_ARG).
+ * Errors: every argument is checked before anything is enqueued; on error nothing is
+ * launched and the status says why. ATTN_ERR_CUDA reports a failed launch. Device-side
+ * waits are bounded (about 2 s); a wait that gives up makes the kernel stop early and
+ * leave a code that attn_debug_error returns as ATTN_ERR_TIMEOUT.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+             int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
+             float scale, int mask_kind, int64_t window, cudaStream_t stream);
+
+/* Options for attn_fwd_ex. Zero-initialise, then set what is needed. */
+typedef struct {
+  uint64_t wait_timeout_ns; /* bound of every device-side wait; 0 = default (2 s) */
+  int inject_stall;         /* test hook: 1 = the loader issues no copies, so every consumer
+                               wait runs out and the kernel exits with ATTN_ERR_TIMEOUT
+                               pending in attn_debug_error; nothing faults or hangs */
+  int grid_ctas;            /* number of persistent CTAs; 0 = one per SM */
+} attn_fwd_options;
+
+/* attn_fwd with options (same arguments, same checks); opts may be NULL. */
+int attn_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse,
+                int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
+                float scale, int mask_kind, int64_t window, cudaStream_t stream,
+                const attn_fwd_options* opts);
+
+/* Human-readable name of an attn_status value (static string, never NULL). */
+const char* attn_status_string(int status);
+
+/*
+ * attn_debug_error: synchronise `stream`, read and clear the device error word of the
+ * current device. Returns ATTN_OK if no device wait gave up since the last call,
+ * ATTN_ERR_TIMEOUT if one did (the raw code, which names the waiting role, goes to
+ * *device_code when device_code is not NULL), ATTN_ERR_CUDA if the synchronisation
+ * itself failed.
+ */
+int attn_debug_error(cudaStream_t stream, int* device_code);
+
+/* Number of persistent work items a launch with these sizes schedules (host-only
+   helper for tests and tools; returns -1 on invalid sizes). */
+int64_t attn_fwd_num_work_items(int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
+                                int mask_kind, int64_t window);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_ATTN_H_ */

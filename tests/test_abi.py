@@ -1,0 +1,99 @@
+"""C-ABI library: loads without a GPU, exports every symbol include/attn.h
+declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_72_b200 import attn as A
+from exact_io_aware_72_b200 import build as BLD
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    BLD.build()
+    return A.load_library()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "attn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|int64_t|const char\*)\s+(attn_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_expected_entry_points():
+    assert declared_functions() == sorted(A.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in A.STATUS.items():
+        assert lib.attn_status_string(code).decode() == name
+    assert lib.attn_status_string(99).decode() == "ATTN_ERR_UNKNOWN"
+
+
+# Fake, never-dereferenced device addresses: far apart, 256-byte aligned.
+Q, K, V, O, L = (0x10000000000 * (i + 1) for i in range(5))
+
+
+def call(lib, q=Q, k=K, v=V, o=O, l=L, B=1, Hq=2, Hkv=2, N=256, d=64, scale=0.125, mask=1, window=0):
+    return lib.attn_fwd(q, k, v, o, l, B, Hq, Hkv, N, d, scale, mask, window, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(k=None), 1), (dict(v=None), 1), (dict(o=None), 1), (dict(l=None), 1),
+    (dict(B=0), 1), (dict(Hq=0), 1), (dict(Hkv=0), 1), (dict(N=0), 1), (dict(B=-3), 1),
+    (dict(Hq=6, Hkv=4), 1), (dict(mask=3), 1), (dict(mask=-1), 1),
+    (dict(mask=2, window=0), 1), (dict(mask=2, window=-5), 1),
+    (dict(scale=0.0), 1), (dict(scale=-0.1), 1), (dict(scale=float("inf")), 1), (dict(scale=float("nan")), 1),
+    (dict(d=32), 2), (dict(d=96), 2), (dict(d=256), 2),
+    (dict(q=Q + 8), 3), (dict(k=K + 4), 3), (dict(v=V + 2), 3), (dict(o=O + 8), 3), (dict(l=L + 2), 3),
+    (dict(o=Q), 1), (dict(o=K + 64), 1), (dict(l=O + 1024), 1), (dict(l=V), 1),
+    (dict(N=(1 << 30) + 1), 1),
+])
+def test_invalid_arguments_rejected_before_launch(lib, kw, status):
+    assert call(lib, **kw) == status
+
+
+def test_valid_arguments_reach_the_device_check(lib):
+    # Everything valid: the next step needs a CUDA device. Without one the call
+    # reports a CUDA error (nothing is launched); with one it would launch.
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    assert call(lib) == 4
+    assert call(lib, mask=2, window=10 ** 9) == 4     # window >= N is accepted (runs as causal)
+
+
+def _items(B, Hq, Hkv, N, mask, window):
+    """Work-item count of the schedule: two 128-row query tiles per item, paired
+    as two heads of one KV group when Hq/Hkv is even, else two blocks of a head."""
+    g = Hq // Hkv
+    mb = -(-N // 128)
+    if g % 2 == 0:
+        return mb * B * Hq // 2
+    return -(-mb // 2) * B * Hq
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 2, 256), (2, 32, 32, 8192), (1, 64, 8, 16384), (1, 32, 8, 131072),
+                                   (1, 32, 32, 131072), (3, 6, 2, 1000), (1, 3, 1, 129), (1, 1, 1, 1)])
+def test_work_item_count(lib, shape):
+    B, Hq, Hkv, N = shape
+    for mask, window in ((0, 0), (1, 0), (2, 4096)):
+        assert lib.attn_fwd_num_work_items(B, Hq, Hkv, N, 128, mask, window) == _items(B, Hq, Hkv, N, mask, window)
+    assert lib.attn_fwd_num_work_items(1, 2, 2, 64, 96, 1, 0) == -1
+    assert lib.attn_fwd_num_work_items(1, 3, 2, 64, 64, 1, 0) == -1
+
+
+def test_python_binding_validates_without_launching():
+    import torch
+    with pytest.raises((TypeError, ValueError)):
+        A.fwd(torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16), torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16),
+              torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16))
