@@ -51,6 +51,25 @@ constexpr float kLn2 = 0.6931471805599453f;
 // bf16 P carry without loss.  The final O / l uses the same max, so the result
 // is unchanged.
 constexpr float kRescaleThreshold = 8.0f;
+// P is packed to bf16 by truncating p * (1 + 2^-9): with the factor folded into
+// the exponent (x + log2(1 + 2^-9)), truncation lands within 3/4 of a bf16 ulp
+// of p (round-to-nearest would be 1/2) at the cost of one byte permute per pair.
+// The factor is common to every p of a row, so O / l is unaffected and the
+// log-sum-exp (from the fp32 sum) subtracts it exactly.
+constexpr float kP16Bias = 0.0028150156f;  // log2(1 + 2^-9)
+// 2^f on [-1/2, 1/2]: degree-3 polynomial with minimal maximum relative error
+// (Remez exchange; csrc/fit_exp2_poly.py), max relative error 7.5e-5, used
+// after Cody-Waite reduction x = n + f for kPolyPairs of every 16 column pairs
+// so that part of the exponentials can run on the FMA pipe instead of the
+// MUFU.  Measured on B200 the softmax loop is bound by instruction issue, not
+// by the MUFU, so the offload is off (0 pairs); it pays only once the MUFU is
+// the limit.
+constexpr float kExp2Poly0 = 0.9999280572f;
+constexpr float kExp2Poly1 = 0.6932609677f;
+constexpr float kExp2Poly2 = 0.2426111251f;
+constexpr float kExp2Poly3 = 0.0551716685f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + M rounds x to an integer in the low bits
+constexpr int kPolyPairs = 0;
 
 enum : int { kMaskFull = 0, kMaskCausal = 1, kMaskWindow = 2 };
 
@@ -426,8 +445,8 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
     const int hi = t ? it.hi[1] : it.hi[0];
     const int row = mblk * kBlockM + row_in_tile;
     float m_run = -INFINITY;
-    float l_run = 0.f;   // sum of P as written (bf16), normalises O
-    float l_lse = 0.f;   // sum of P in fp32, for the log-sum-exp
+    float l_run = 0.f;   // row sum of P as written (bf16), normalises O
+    float l_lse = 0.f;   // fp32 row sum of p (carries the kP16Bias factor)
     // Both softmax warpgroups walk the item's whole KV range so they can hand
     // the turn token back and forth: the exp loop of one tile runs while
     // the tensor core works on the other tile (the exp unit is the shared
@@ -485,13 +504,19 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
         ++turn_cnt;
       }
       if (active) {
-        // p = 2^(s*c - m) on column pairs (packed fp32 FMA), then P to bf16 by
-        // rounding half up on the integer pipe (the fp32->bf16 convert would
-        // share the exp2 unit).  O is normalised by the sum of exactly these
-        // rounded values, so each row's weights stay a convex combination; the
-        // log-sum-exp uses the fp32 sum.  P goes to TMEM 16 columns at a time.
+        // p = 2^(s*c - m) on column pairs (packed fp32 FMA); the first
+        // kPolyPairs pairs of every 16 use the polynomial on the FMA pipe, the
+        // rest the MUFU ex2.  P goes to TMEM 16 columns at a time.  O is
+        // normalised by the sum of exactly the bf16 values written (so a row
+        // dominated by one key returns that key's v); the log-sum-exp uses the
+        // fp32 sum of p.
         const uint64_t c2 = f32x2_pack(c, c);
-        const uint64_t nb2 = f32x2_pack(neg_base, neg_base);
+        const uint64_t nb2 = f32x2_pack(neg_base + kP16Bias, neg_base + kP16Bias);
+        const uint64_t magic2 = f32x2_pack(kRoundMagic, kRoundMagic);
+        const uint64_t nmagic2 = f32x2_pack(-kRoundMagic, -kRoundMagic);
+        const uint64_t neg1 = f32x2_pack(-1.f, -1.f);
+        const uint64_t q3 = f32x2_pack(kExp2Poly3, kExp2Poly3), q2 = f32x2_pack(kExp2Poly2, kExp2Poly2);
+        const uint64_t q1 = f32x2_pack(kExp2Poly1, kExp2Poly1), q0 = f32x2_pack(kExp2Poly0, kExp2Poly0);
         uint64_t so2 = 0, sl2 = 0;  // (+0.f, +0.f)
 #pragma unroll
         for (int chunk = 0; chunk < 4; ++chunk) {
@@ -505,14 +530,31 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int e = chunk * 32 + 2 * i;
-            float x0, x1;
-            f32x2_unpack(f32x2_fma(f32x2_pack(s[e], s[e + 1]), c2, nb2), x0, x1);
-            const float p0 = fast_exp2(x0);
-            const float p1 = fast_exp2(x1);
-            const uint32_t u0 = __float_as_uint(p0) + 0x8000u;
-            const uint32_t u1 = __float_as_uint(p1) + 0x8000u;
-            pk[i] = __byte_perm(u0, u1, 0x7632);
-            so2 = f32x2_add(so2, f32x2_pack(__uint_as_float(u0 & 0xffff0000u), __uint_as_float(u1 & 0xffff0000u)));
+            const uint64_t x2 = f32x2_fma(f32x2_pack(s[e], s[e + 1]), c2, nb2);
+            float x0, x1, p0, p1;
+            f32x2_unpack(x2, x0, x1);
+            if (i < kPolyPairs) {
+              // 2^x = 2^n q(f): n = round(x) via the magic constant, f = x - n,
+              // q by Horner, n added to the exponent field.  x is clamped at
+              // -125 so masked (-inf) entries give 2^-125 q(f), not garbage.
+              const uint64_t xc = f32x2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+              const uint64_t t2 = f32x2_add(xc, magic2);
+              const uint64_t f2 = f32x2_fma(f32x2_add(t2, nmagic2), neg1, xc);
+              uint64_t r2 = f32x2_fma(f2, q3, q2);
+              r2 = f32x2_fma(f2, r2, q1);
+              r2 = f32x2_fma(f2, r2, q0);
+              float r0, r1, t0, t1;
+              f32x2_unpack(r2, r0, r1);
+              f32x2_unpack(t2, t0, t1);
+              p0 = __uint_as_float(__float_as_uint(r0) + (__float_as_uint(t0) << 23));
+              p1 = __uint_as_float(__float_as_uint(r1) + (__float_as_uint(t1) << 23));
+            } else {
+              p0 = fast_exp2(x0);
+              p1 = fast_exp2(x1);
+            }
+            pk[i] = __byte_perm(__float_as_uint(p0), __float_as_uint(p1), 0x7632);  // truncate to bf16x2
+            so2 = f32x2_add(so2, f32x2_pack(__uint_as_float(__float_as_uint(p0) & 0xffff0000u),
+                                            __uint_as_float(__float_as_uint(p1) & 0xffff0000u)));
             sl2 = f32x2_add(sl2, f32x2_pack(p0, p1));
           }
           tmem_store_16cols(tS + chunk * 16, pk);
@@ -569,7 +611,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
             dst[cc * 4 + v] = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
         }
       }
-      if (row_ok) p.lse[head_row] = (m_run + __log2f(l_lse)) * kLn2;
+      if (row_ok) p.lse[head_row] = (m_run + __log2f(l_lse) - kP16Bias) * kLn2;
     }
     tc_fence_before_sync();
     __syncwarp();
