@@ -339,10 +339,20 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="dense")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--shape", default=None,
+                    help="B,Hq,Hkv,N,d: run this shape instead of a named workload (profiling sweeps)")
+    ap.add_argument("--mask", choices=["full", "causal", "sliding_window"], default=None)
+    ap.add_argument("--window", type=int, default=None)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
+    if args.shape or args.mask:
+        from dataclasses import replace
+        B, Hq, Hkv, N, d = (int(x) for x in args.shape.split(",")) if args.shape else (w.B, w.Hq, w.Hkv, w.N, w.d)
+        mask = args.mask or w.mask
+        w = replace(w, name="custom", B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, mask=mask,
+                    window=args.window if mask == "sliding_window" else None, sharp=False)
     if args.impl == "reference":
         run_reference(args, w)
     else:

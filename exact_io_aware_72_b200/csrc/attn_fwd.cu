@@ -94,7 +94,7 @@ struct Plan {
   int mask_kind;
   int64_t window;
   int pair_heads;
-  int64_t num_mblk, row_units, head_units, num_items;
+  int64_t num_mblk, row_units, head_units, num_items, super_items;
 };
 
 // Checks that need no device; fills the schedule plan.
@@ -122,6 +122,7 @@ int check_sizes(int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d, int ma
   plan.row_units = plan.pair_heads ? plan.num_mblk : (plan.num_mblk + 1) / 2;
   plan.head_units = plan.pair_heads ? B * Hq / 2 : B * Hq;
   plan.num_items = plan.row_units * plan.head_units;
+  plan.super_items = plan.head_units * ((plan.row_units + 1) / 2);  // row units r and R-1-r together
   if (plan.num_items > 0x7fffffff) return ATTN_ERR_INVALID_ARG;
   return ATTN_OK;
 }
@@ -213,7 +214,7 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* out, float* l
 
   int grid = info.sm_count;
   if (opts && opts->grid_ctas > 0) grid = opts->grid_ctas;
-  if (grid > p.num_items) grid = p.num_items;
+  if (grid > plan.super_items) grid = static_cast<int>(plan.super_items);
 
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));

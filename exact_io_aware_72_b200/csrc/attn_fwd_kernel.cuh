@@ -90,9 +90,9 @@ struct FwdParams {
   float scale_log2;  // scale * log2(e)
   int pair_heads;    // 1: the two tiles are two heads of one KV group
   int num_mblk;      // ceil(N / 128)
-  int row_units;     // query-block units per head (unit = block or block pair)
-  int head_units;    // items per row unit
-  int num_items;
+  int row_units;     // row units per head unit (unit = one block, or a pair of blocks)
+  int head_units;    // (b, head) or (b, head pair) units
+  int num_items;     // row_units * head_units
   unsigned long long timeout_ns;
   int inject_stall;
 };
@@ -147,21 +147,21 @@ __device__ __forceinline__ void kv_range(const FwdParams& p, int m, int& lo, int
   }
 }
 
-// Items are ordered longest first (row unit descending), heads inside.
-__device__ __forceinline__ WorkItem decode_item(const FwdParams& p, int idx) {
+// Work item (head unit hu, row unit r): head unit = (b, query head) or
+// (b, query-head pair); row unit = one 128-row block (head pairs) or a pair of
+// consecutive blocks of one head.
+__device__ __forceinline__ WorkItem decode_item(const FwdParams& p, int hu, int r) {
   WorkItem it;
-  const int r = p.row_units - 1 - idx / p.head_units;
-  const int u = idx % p.head_units;
   if (p.pair_heads) {
     const int hpairs = p.Hq >> 1;
-    it.b = u / hpairs;
-    const int hp = u - it.b * hpairs;
+    it.b = hu / hpairs;
+    const int hp = hu - it.b * hpairs;
     it.head[0] = 2 * hp;
     it.head[1] = 2 * hp + 1;
     it.mblk[0] = it.mblk[1] = r;
   } else {
-    it.b = u / p.Hq;
-    it.head[0] = it.head[1] = u - it.b * p.Hq;
+    it.b = hu / p.Hq;
+    it.head[0] = it.head[1] = hu - it.b * p.Hq;
     it.mblk[0] = 2 * r;
     it.mblk[1] = 2 * r + 1;
   }
@@ -192,19 +192,36 @@ __device__ __forceinline__ bool tile_is_partial(const FwdParams& p, int m, int j
   return partial;
 }
 
-// Static persistent schedule: round k hands item k*G + c (even k) or
-// k*G + G-1-c (odd k) to CTA c, pairing heavy items with light ones.
+// Static persistent schedule without any shared counter.  Row units r and
+// R-1-r of one head form a super-item: under a causal mask their costs add up
+// to the same total for every r, so dealing super-items round-robin (CTA c
+// takes c, c+G, c+2G, ...) balances the load.  Super-items are numbered head
+// unit by head unit, so the CTAs running at any moment share a few heads' K/V
+// through L2 instead of each streaming its own head from HBM.
 struct Schedule {
-  int k, cta, grid, total;
-  __device__ Schedule(int cta_, int grid_, int total_) : k(0), cta(cta_), grid(grid_), total(total_) {}
-  __device__ __forceinline__ bool next(int& idx) {
-    while (true) {
-      const int base = k * grid;
-      if (base >= total) return false;
-      idx = base + ((k & 1) ? (grid - 1 - cta) : cta);
-      ++k;
-      if (idx < total) return true;
+  int g, sub, grid, total, per_head, R;
+  __device__ Schedule(const FwdParams& p, int cta, int grid_)
+      : g(cta), sub(0), grid(grid_), per_head((p.row_units + 1) >> 1), R(p.row_units) {
+    total = p.head_units * per_head;
+  }
+  // Next work item of this CTA (long row unit first); false when done.
+  __device__ __forceinline__ bool next(int& hu, int& r) {
+    if (g >= total) return false;
+    hu = g / per_head;
+    const int s = g - hu * per_head;
+    if (sub == 0) {
+      r = R - 1 - s;
+      if (r == s) {
+        g += grid;
+      } else {
+        sub = 1;
+      }
+    } else {
+      r = s;
+      sub = 0;
+      g += grid;
     }
+    return true;
   }
 };
 
@@ -268,10 +285,10 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sbase
   uint32_t q_issued = 0;
   int items = 0;
   bool ok = !p.inject_stall;
-  Schedule sched(blockIdx.x, gridDim.x, p.num_items);
-  int idx;
-  while (ok && sched.next(idx)) {
-    const WorkItem it = decode_item(p, idx);
+  Schedule sched(p, blockIdx.x, gridDim.x);
+  int hu, r;
+  while (ok && sched.next(hu, r)) {
+    const WorkItem it = decode_item(p, hu, r);
     if (items > 0 && !w.wait(bar(L::kQEmpty), (items - 1) & 1, (kRoleProducer << 8) | L::kQEmpty)) {
       ok = false;
       break;
@@ -344,10 +361,10 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
   uint32_t p_cnt = 0;
   int items = 0;
   bool ok = true;
-  Schedule sched(blockIdx.x, gridDim.x, p.num_items);
-  int idx;
-  while (ok && sched.next(idx)) {
-    const WorkItem it = decode_item(p, idx);
+  Schedule sched(p, blockIdx.x, gridDim.x);
+  int hu, r;
+  while (ok && sched.next(hu, r)) {
+    const WorkItem it = decode_item(p, hu, r);
     const int valid = t ? it.valid[1] : it.valid[0];
     const int lo = t ? it.lo[1] : it.lo[0];
     const int hi = t ? it.hi[1] : it.hi[0];
@@ -433,10 +450,10 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
   uint32_t turn_cnt = 0;
   int items = 0;
   bool ok = true;
-  Schedule sched(blockIdx.x, gridDim.x, p.num_items);
-  int idx;
-  while (ok && sched.next(idx)) {
-    const WorkItem it = decode_item(p, idx);
+  Schedule sched(p, blockIdx.x, gridDim.x);
+  int hu, r;
+  while (ok && sched.next(hu, r)) {
+    const WorkItem it = decode_item(p, hu, r);
     // This warp's tile, picked with selects so the item stays in registers.
     const int mblk = t ? it.mblk[1] : it.mblk[0];
     const int head = t ? it.head[1] : it.head[0];
