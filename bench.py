@@ -42,7 +42,9 @@ KERNEL_SOURCES = ["exact_io_aware_72_b200/csrc/attn_fwd.cu", "exact_io_aware_72_
 # DRAM bytes per launch of the forward kernel from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the kernel
 # sources it was taken on; reported only while the sources still match.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    ("dense", "62f2fcd30acce73a"): 405841152 + 107980800,   # profiles/attn_fwd_dense_ncu.md
+}
 
 
 def visible_pairs(N: int, mask: str, window) -> int:
