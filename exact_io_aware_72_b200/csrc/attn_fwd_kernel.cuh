@@ -10,7 +10,7 @@
 //   warps 0-3   softmax for query tile 0 (thread = one query row = one TMEM lane)
 //   warps 4-7   softmax for query tile 1
 //   warp  8     TMA loader: Q tiles once per work item, K/V tiles through a ring
-//   warps 9-10  tcgen05 issuers, one thread per query tile: S = Q K^T and
+//   warps 9-10  tcgen05 issuers, one warp per query tile: S = Q K^T and
 //               O += P V; warp 9 also owns the TMEM allocation
 //   warp  11    idle
 // Registers: launched at 168 per thread; the softmax warpgroups raise theirs to
@@ -335,11 +335,13 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sbase
   if (q_issued > 0) w.drain(bar(L::kQFull), (q_issued - 1) & 1, (kRoleProducer << 8) | L::kQFull);
 }
 
-// One issuing thread per query tile t.  For each KV tile j of the item:
+// One issuing warp per query tile t: all lanes run the loop with warp-uniform
+// values (descriptor arithmetic stays on the uniform datapath) and one elected
+// lane issues each tcgen05 instruction.  For each KV tile j of the item:
 //   O_t += P_t(j-1) V_{j-1}   (once the softmax has written P_t(j-1))
 //   S_t  = Q_t K_j^T          (after that P V in issue order, since P aliases S)
-// and releases K_j / V_{j-1} / Q with commits; the other tile's thread does the
-// same, so each ring slot is freed after both threads' reads complete.
+// and releases K_j / V_{j-1} / Q with commits; the other tile's warp does the
+// same, so each ring slot is freed after both warps' reads complete.
 template <int D>
 __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tmem, const Waiter& w,
                                          int t) {
@@ -356,6 +358,11 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
   const uint64_t k_desc0 = smem_desc_sw128(sbase + L::kKVOff, 16, 1024);
   const uint64_t v_desc0 = smem_desc_sw128(sbase + L::kKVOff, L::kChunkBytes, 1024);
   const int code = (kRoleMma << 8) | (t << 7);
+  // Every lane waits; the warp proceeds only if all lanes saw the phase.
+  auto wait_all = [&](uint32_t b, uint32_t parity, int c) -> bool {
+    const bool got = w.wait(b, parity, c);
+    return __all_sync(0xffffffffu, got);
+  };
 
   uint32_t kv_n = 0;
   uint32_t p_cnt = 0;
@@ -368,25 +375,25 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
     const int valid = t ? it.valid[1] : it.valid[0];
     const int lo = t ? it.lo[1] : it.lo[0];
     const int hi = t ? it.hi[1] : it.hi[0];
-    if (!w.wait(bar(L::kQFull), items & 1, code | L::kQFull)) break;
+    if (!wait_all(bar(L::kQFull), items & 1, code | L::kQFull)) break;
     tc_fence_after_sync();
     bool pend = false;
     bool first_pv = true;
 
     // O_t += P_t V for the V tile with load index vn.
     auto issue_pv = [&](uint32_t vn) -> bool {
-      if (first_pv && items > 0 && !w.wait(bar(L::kOFree + t), (items - 1) & 1, code | (L::kOFree + t)))
+      if (first_pv && items > 0 && !wait_all(bar(L::kOFree + t), (items - 1) & 1, code | (L::kOFree + t)))
         return false;
-      if (!w.wait(bar(L::kPFull + t), p_cnt & 1, code | (L::kPFull + t))) return false;
+      if (!wait_all(bar(L::kPFull + t), p_cnt & 1, code | (L::kPFull + t))) return false;
       ++p_cnt;
       const uint32_t vslot = vn % L::kStages;
-      if (!w.wait(bar(L::kKVFull + vslot), (vn / L::kStages) & 1, code | (L::kKVFull + vslot))) return false;
+      if (!wait_all(bar(L::kKVFull + vslot), (vn / L::kStages) & 1, code | (L::kKVFull + vslot))) return false;
       tc_fence_after_sync();
       const uint64_t vd = v_desc0 + ((vslot * L::kTileBytes) >> 4);
 #pragma unroll
       for (int kk = 0; kk < kBlockN / 16; ++kk) {
         // 16 keys = two 8-row swizzle atoms = 2048 B further into the V tile.
-        mma_bf16_ts(o_tmem, s_tmem + kk * 8, vd + ((kk * 2048) >> 4), idesc_o, (kk > 0 || !first_pv) ? 1u : 0u);
+        mma_bf16_ts_elect(o_tmem, s_tmem + kk * 8, vd + ((kk * 2048) >> 4), idesc_o, (kk > 0 || !first_pv) ? 1u : 0u);
       }
       first_pv = false;
       pend = false;
@@ -399,7 +406,7 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
         ok = false;
         break;
       }
-      if (!w.wait(bar(L::kKVFull + kslot), (kv_n / L::kStages) & 1, code | (L::kKVFull + kslot))) {
+      if (!wait_all(bar(L::kKVFull + kslot), (kv_n / L::kStages) & 1, code | (L::kKVFull + kslot))) {
         ok = false;
         break;
       }
@@ -411,25 +418,25 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
           // K-major operands: 16 elements = 32 B inside a 128 B swizzled row,
           // the next 64 columns 16 KB further.
           const uint32_t off = ((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4;
-          mma_bf16_ss(s_tmem, q_desc + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
+          mma_bf16_ss_elect(s_tmem, q_desc + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(L::kSFull + t));
+        tc_commit_elect(bar(L::kSFull + t));
         pend = true;
       }
-      tc_commit(bar(L::kKVEmpty + kslot));                                   // K_j read
-      if (j > it.lo_u) tc_commit(bar(L::kKVEmpty + (kv_n - 1) % L::kStages));  // V_{j-1} read
-      if (j == it.hi_u) tc_commit(bar(L::kQEmpty));                          // Q read
+      tc_commit_elect(bar(L::kKVEmpty + kslot));                                   // K_j read
+      if (j > it.lo_u) tc_commit_elect(bar(L::kKVEmpty + (kv_n - 1) % L::kStages));  // V_{j-1} read
+      if (j == it.hi_u) tc_commit_elect(bar(L::kQEmpty));                          // Q read
       kv_n += 2;
     }
     if (!ok) break;
     if (pend && !issue_pv(kv_n - 1)) break;
-    tc_commit(bar(L::kKVEmpty + (kv_n - 1) % L::kStages));  // V_hi read
-    if (first_pv && items > 0 && !w.wait(bar(L::kOFree + t), (items - 1) & 1, code | (L::kOFree + t))) break;
-    tc_commit(bar(L::kODone + t));
+    tc_commit_elect(bar(L::kKVEmpty + (kv_n - 1) % L::kStages));  // V_hi read
+    if (first_pv && items > 0 && !wait_all(bar(L::kOFree + t), (items - 1) & 1, code | (L::kOFree + t))) break;
+    tc_commit_elect(bar(L::kODone + t));
     ++items;
   }
   // Drain: every MMA this thread issued must complete before TMEM is freed.
-  tc_commit(bar(L::kFin + t));
+  tc_commit_elect(bar(L::kFin + t));
   w.drain(bar(L::kFin + t), 0, code | (L::kFin + t));
 }
 
@@ -690,8 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     if (lane == 0) producer_role<D>(p, sbase, w);
     __syncwarp();
   } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
-    if (lane == 0) mma_role<D>(p, sbase, tmem, w, warp - kMmaWarp);
-    __syncwarp();
+    mma_role<D>(p, sbase, tmem, w, warp - kMmaWarp);
   }
 
   tc_fence_before_sync();
