@@ -47,10 +47,13 @@ constexpr uint32_t kOtherRegs = 88;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * 168, "register split exceeds launch");
 constexpr float kLn2 = 0.6931471805599453f;
 // The running max is only moved when a row's max grows by more than this many
-// powers of two; until then P may exceed 1 by up to 2^8, which fp32 sums and
-// bf16 P carry without loss.  The final O / l uses the same max, so the result
-// is unchanged.
-constexpr float kRescaleThreshold = 8.0f;
+// powers of two; until then P may exceed 1 by up to 2^32.  bf16 P and fp32 sums
+// and accumulators carry that without loss (relative precision does not depend
+// on scale; a row sum stays below 2^32 * 2^17 keys = 2^49), and the final O / l
+// and log-sum-exp use the same max, so the result is unchanged.  A large margin
+// keeps O rescales (a TMEM round trip on the softmax critical path) rare even
+// for rows whose scores keep growing.
+constexpr float kRescaleThreshold = 32.0f;
 // P is packed to bf16 by truncating p * (1 + 2^-9): with the factor folded into
 // the exponent (x + log2(1 + 2^-9)), truncation lands within 3/4 of a bf16 ulp
 // of p (round-to-nearest would be 1/2) at the cost of one byte permute per pair.
