@@ -211,6 +211,7 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* out, float* l
   p.num_items = static_cast<int>(plan.num_items);
   p.timeout_ns = (opts && opts->wait_timeout_ns) ? opts->wait_timeout_ns : kDefaultTimeoutNs;
   p.inject_stall = (opts && opts->inject_stall) ? 1 : 0;
+  p.out_v8 = (reinterpret_cast<uintptr_t>(out) % 32 == 0) ? 1 : 0;
 
   int grid = info.sm_count;
   if (opts && opts->grid_ctas > 0) grid = opts->grid_ctas;

@@ -73,6 +73,9 @@ constexpr float kExp2Poly2 = 0.2426111251f;
 constexpr float kExp2Poly3 = 0.0551716685f;
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + M rounds x to an integer in the low bits
 constexpr int kPolyPairs = 0;
+// Steps before the end of a work item at which the loader prefetches the next
+// item's first tiles into L2 (each step is a few microseconds of work).
+constexpr int kPrefetchSteps = 6;
 
 enum : int { kMaskFull = 0, kMaskCausal = 1, kMaskWindow = 2 };
 
@@ -98,6 +101,7 @@ struct FwdParams {
   int num_items;     // row_units * head_units
   unsigned long long timeout_ns;
   int inject_stall;
+  int out_v8;        // 1: out is 32-byte aligned, rows are written with 32-byte stores
 };
 
 template <int D>
@@ -274,6 +278,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // ------------------------------------------------------------ roles
+// L2 prefetch of the next work item's Q tiles and of its first two K/V tiles
+// (sched has already moved past the current item).
+template <int D>
+__device__ __forceinline__ void prefetch_next_item(const FwdParams& p, Schedule sched) {
+  int hu, r;
+  if (!sched.next(hu, r)) return;
+  const WorkItem n = decode_item(p, hu, r);
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+      if (n.valid[t]) tma_prefetch_3d(&p.tm_q, c * 64, n.mblk[t] * kBlockM, n.b * p.Hq + n.head[t]);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      if (n.lo_u + j > n.hi_u) break;
+      tma_prefetch_3d(&p.tm_k, c * 64, (n.lo_u + j) * kBlockN, n.b * p.Hkv + n.hkv);
+      tma_prefetch_3d(&p.tm_v, c * 64, (n.lo_u + j) * kBlockN, n.b * p.Hkv + n.hkv);
+    }
+  }
+}
+
 template <int D>
 __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sbase, const Waiter& w) {
   using L = SmemLayout<D>;
@@ -292,22 +317,31 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sbase
   int hu, r;
   while (ok && sched.next(hu, r)) {
     const WorkItem it = decode_item(p, hu, r);
-    if (items > 0 && !w.wait(bar(L::kQEmpty), (items - 1) & 1, (kRoleProducer << 8) | L::kQEmpty)) {
-      ok = false;
-      break;
-    }
-    const uint32_t qbytes = (it.valid[0] + it.valid[1]) * L::kTileBytes;
-    mbar_arrive_expect_tx(bar(L::kQFull), qbytes);
-    ++q_issued;
+    // Q of this item goes into the single Q buffer once the previous item's
+    // last S has read it.  The item's first K and V tiles are issued before
+    // that wait (their ring slots free up earlier), so they are already in
+    // flight while the previous item drains.
+    auto load_q = [&]() -> bool {
+      if (items > 0 && !w.wait(bar(L::kQEmpty), (items - 1) & 1, (kRoleProducer << 8) | L::kQEmpty)) return false;
+      const uint32_t qbytes = (it.valid[0] + it.valid[1]) * L::kTileBytes;
+      mbar_arrive_expect_tx(bar(L::kQFull), qbytes);
+      ++q_issued;
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      if (!it.valid[t]) continue;
+      for (int t = 0; t < 2; ++t) {
+        if (!it.valid[t]) continue;
 #pragma unroll
-      for (int c = 0; c < L::kChunks; ++c)
-        tma_load_3d(sbase + L::kQOff + t * L::kTileBytes + c * L::kChunkBytes, &p.tm_q, bar(L::kQFull),
-                    c * 64, it.mblk[t] * kBlockM, it.b * p.Hq + it.head[t], pol_q);
-    }
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(sbase + L::kQOff + t * L::kTileBytes + c * L::kChunkBytes, &p.tm_q, bar(L::kQFull),
+                      c * 64, it.mblk[t] * kBlockM, it.b * p.Hq + it.head[t], pol_q);
+      }
+      return true;
+    };
+    // A few steps before the item ends, start pulling what the next item
+    // reads first (its Q tiles and first K/V tiles) into L2, so the next
+    // item's loads do not wait on DRAM.
+    const int pf_step = max(it.lo_u, it.hi_u - kPrefetchSteps);
     for (int j = it.lo_u; j <= it.hi_u && ok; ++j) {
+      if (j == pf_step) prefetch_next_item<D>(p, sched);
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
         const uint32_t slot = kv_n % L::kStages;
@@ -324,6 +358,10 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sbase
           tma_load_3d(sbase + L::kKVOff + slot * L::kTileBytes + c * L::kChunkBytes, map,
                       bar(L::kKVFull + slot), c * 64, j * kBlockN, it.b * p.Hkv + it.hkv, pol_kv);
         ++kv_n;
+        if (j == it.lo_u && kv == 1 && !load_q()) {
+          ok = false;
+          break;
+        }
       }
     }
     ++items;
@@ -405,11 +443,13 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
 
     for (int j = it.lo_u; j <= it.hi_u; ++j) {
       const uint32_t kslot = kv_n % L::kStages;
-      if (pend && !issue_pv(kv_n - 1)) {
+      // K_j is normally resident long before P_t(j-1) is ready; confirming it
+      // first lets P V and the next S issue back to back once P arrives.
+      if (!wait_all(bar(L::kKVFull + kslot), (kv_n / L::kStages) & 1, code | (L::kKVFull + kslot))) {
         ok = false;
         break;
       }
-      if (!wait_all(bar(L::kKVFull + kslot), (kv_n / L::kStages) & 1, code | (L::kKVFull + kslot))) {
+      if (pend && !issue_pv(kv_n - 1)) {
         ok = false;
         break;
       }
@@ -624,6 +664,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
       const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
       const size_t head_row = (static_cast<size_t>(it.b) * p.Hq + head) * p.N + (row_ok ? row : 0);
       uint4* dst = reinterpret_cast<uint4*>(p.out + head_row * D);
+      const uint64_t inv2 = f32x2_pack(inv_l, inv_l);
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -631,11 +672,23 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
         if (row_ok) {
           uint32_t h[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            h[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+          for (int i = 0; i < 16; ++i) {
+            float a, b;
+            f32x2_unpack(f32x2_mul(f32x2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), inv2), a, b);
+            h[i] = pack_bf16x2(a, b);
+          }
+          // 32 columns = 64 bytes of the row: two 32-byte stores when the
+          // output allows it (fewer store instructions and L1 wavefronts).
+          if (p.out_v8) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[cc * 4 + v] = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+            for (int v = 0; v < 2; ++v)
+              st_global_v8(dst + cc * 4 + 2 * v, h[8 * v], h[8 * v + 1], h[8 * v + 2], h[8 * v + 3], h[8 * v + 4],
+                           h[8 * v + 5], h[8 * v + 6], h[8 * v + 7]);
+          } else {
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[cc * 4 + v] = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+          }
         }
       }
       if (row_ok) p.lse[head_row] = (m_run + __log2f(l_lse) - kP16Bias) * kLn2;

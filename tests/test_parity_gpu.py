@@ -97,3 +97,18 @@ def test_outputs_fully_overwritten(cuda_ok):
     fwd(q, k, v, mask="causal", out=out, lse=lse)
     torch.cuda.synchronize()
     assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+
+
+def test_out_16_byte_aligned_matches_32_byte_aligned_bitwise(cuda_ok):
+    # Rows of out are written with 32-byte stores when out is 32-byte aligned
+    # and with 16-byte stores otherwise; both paths must give the same bits.
+    from exact_io_aware_72_b200 import fwd
+    q, k, v = (t.cuda() for t in make_qkv(1, 4, 2, 333, 128, 26))
+    o_ref, l_ref = run_cuda(q, k, v, "causal")
+    buf = torch.empty(q.numel() + 8, dtype=q.dtype, device=q.device)
+    out = buf[8:].view(q.shape)  # 16 bytes past a 256-byte boundary
+    assert out.data_ptr() % 32 == 16
+    lse = torch.empty_like(l_ref)
+    fwd(q, k, v, mask="causal", out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.equal(out, o_ref) and torch.equal(lse, l_ref)
