@@ -204,16 +204,34 @@ __device__ __forceinline__ bool tile_is_partial(const FwdParams& p, int m, int j
 // to the same total for every r, so dealing super-items round-robin (CTA c
 // takes c, c+G, c+2G, ...) balances the load.  Super-items are numbered head
 // unit by head unit, so the CTAs running at any moment share a few heads' K/V
-// through L2 instead of each streaming its own head from HBM.
+// through L2 instead of each streaming its own head from HBM.  When the last,
+// partial round has at most G/2 super-items, they are dealt as single row
+// units instead (CTA c takes unit c of them), which halves that round's length.
 struct Schedule {
   int g, sub, grid, total, per_head, R;
+  int split_from;  // first super-item of the split last round (total if none)
+  int tail;        // this CTA's row unit in the split round, -1 if none / taken
   __device__ Schedule(const FwdParams& p, int cta, int grid_)
       : g(cta), sub(0), grid(grid_), per_head((p.row_units + 1) >> 1), R(p.row_units) {
     total = p.head_units * per_head;
+    const int rem = total % grid;
+    const bool split = rem > 0 && 2 * rem <= grid;
+    split_from = split ? total - rem : total;
+    tail = (split && cta < 2 * rem) ? cta : -1;
   }
   // Next work item of this CTA (long row unit first); false when done.
   __device__ __forceinline__ bool next(int& hu, int& r) {
-    if (g >= total) return false;
+    if (g >= split_from) {
+      if (tail < 0) return false;
+      const int sidx = split_from + (tail >> 1);
+      hu = sidx / per_head;
+      const int s = sidx - hu * per_head;
+      const bool second = (tail & 1) != 0;
+      tail = -1;
+      if (second && R - 1 - s == s) return false;  // middle unit of an odd R: one item only
+      r = second ? s : R - 1 - s;
+      return true;
+    }
     hu = g / per_head;
     const int s = g - hu * per_head;
     if (sub == 0) {
