@@ -605,12 +605,6 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
         uint64_t so2 = 0, sl2 = 0;  // (+0.f, +0.f)
 #pragma unroll
         for (int chunk = 0; chunk < 4; ++chunk) {
-          if (chunk == 3) {
-            // Hand the turn over one chunk early: the other tile's wake-up
-            // overlaps the tail of this loop.
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::kTurn + (t ^ 1)));
-          }
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -669,7 +663,12 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
         tmem_store_wait();
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::kPFull + t));
+        if (lane == 0) {
+          mbar_arrive(bar(L::kPFull + t));
+          // Hand the turn to the other tile once P is published: its exp loop
+          // then runs while the tensor core takes this tile's P V and next S.
+          mbar_arrive(bar(L::kTurn + (t ^ 1)));
+        }
       }
     }
     if (!ok) break;
