@@ -319,6 +319,7 @@ def run_ours(args, w):
                          "peak_source": f"{peak_src} bf16_tflops (burst)",
                          "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak))},
             "gpu_launches": args.steps,
+            "launch_ms": {"median": statistics.median(per_launch_ms), "best": min(per_launch_ms)},
             "clocks": clk,
             "e2e": {"value": world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
