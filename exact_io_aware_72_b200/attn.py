@@ -18,7 +18,8 @@ STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3:
           4: "ATTN_ERR_CUDA", 5: "ATTN_ERR_TIMEOUT"}
 ATTN_ERR_TIMEOUT = 5
 LIB_NAME = "libattn_b200.so"
-EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_status_string", "attn_debug_error", "attn_fwd_num_work_items")
+EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_status_string", "attn_debug_error", "attn_fwd_num_work_items",
+           "attn_bwd", "attn_bwd_ex", "attn_bwd_workspace_bytes", "attn_bwd_debug_error")
 
 _lib = None
 
@@ -59,6 +60,15 @@ def load_library():
     lib.attn_debug_error.restype = ctypes.c_int
     lib.attn_fwd_num_work_items.argtypes = [i64, i64, i64, i64, i64, ctypes.c_int, i64]
     lib.attn_fwd_num_work_items.restype = i64
+    bwd_args = [vp] * 10 + [ctypes.c_size_t, i64, i64, i64, i64, i64, ctypes.c_float, ctypes.c_int, i64, vp]
+    lib.attn_bwd.argtypes = bwd_args
+    lib.attn_bwd.restype = ctypes.c_int
+    lib.attn_bwd_ex.argtypes = bwd_args + [ctypes.POINTER(FwdOptions)]
+    lib.attn_bwd_ex.restype = ctypes.c_int
+    lib.attn_bwd_workspace_bytes.argtypes = [i64, i64, i64]
+    lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_bwd_debug_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    lib.attn_bwd_debug_error.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -110,6 +120,68 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float
     if st != 0:
         raise AttnError(st, "attn_fwd")
     return out, lse
+
+
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
+        dout: torch.Tensor, scale: Optional[float] = None, mask: str = "causal", window: Optional[int] = None,
+        dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
+        workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+        wait_timeout_ns: int = 0, grid_ctas: int = 0) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Exact attention backward: returns (dq, dk, dv), the gradients of
+    sum(dout * out) for the forward's q, k, v (same scale / mask / window).
+
+    ``out`` and ``lse`` are the forward's outputs for these inputs. The fp32
+    workspace (B*Hq*N floats, allocated here when not given) holds the row
+    terms D = rowsum(dout * out) between the kernels of this call.
+    """
+    lib = load_library()
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _check(t, name, torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    B, Hq, N, d = q.shape
+    Bk, Hkv, Nk, dk_ = k.shape
+    if (Bk, Nk, dk_) != (B, N, d) or tuple(v.shape) != tuple(k.shape) or out.shape != q.shape \
+            or dout.shape != q.shape or tuple(lse.shape) != (B, Hq, N):
+        raise ValueError("q, k, v, out, lse, dout shapes disagree")
+    if mask not in MASKS:
+        raise ValueError(f"mask must be one of {sorted(MASKS)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, name, ref in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+        _check(t, name, torch.bfloat16, 4)
+        if t.shape != ref.shape:
+            raise ValueError(f"{name} has the wrong shape")
+    ws_bytes = int(lib.attn_bwd_workspace_bytes(B, Hq, N))
+    if workspace is None:
+        workspace = torch.empty(ws_bytes // 4, dtype=torch.float32, device=q.device)
+    if not (workspace.is_cuda and workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    opts = FwdOptions(int(wait_timeout_ns), 0, int(grid_ctas))
+    with torch.cuda.device(q.device):
+        st = lib.attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                             dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), B, Hq, Hkv, N, d, float(scale),
+                             MASKS[mask], int(window) if window is not None else 0,
+                             ctypes.c_void_p(stream.cuda_stream), ctypes.byref(opts))
+    if st != 0:
+        raise AttnError(st, "attn_bwd")
+    return dq, dk, dv
+
+
+def bwd_debug_error(stream: Optional[torch.cuda.Stream] = None, device=None) -> Tuple[int, int]:
+    """Synchronise and read/clear the backward kernels' error word: (status, raw code)."""
+    lib = load_library()
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    code = ctypes.c_int(0)
+    with torch.cuda.device(stream.device):
+        st = lib.attn_bwd_debug_error(ctypes.c_void_p(stream.cuda_stream), ctypes.byref(code))
+    return st, code.value
 
 
 def debug_error(stream: Optional[torch.cuda.Stream] = None, device=None) -> Tuple[int, int]:

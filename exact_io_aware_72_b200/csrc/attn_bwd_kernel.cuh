@@ -1,0 +1,721 @@
+// Exact attention backward for sm_100a: the gradients of sum(dO * O) with
+// respect to q, k and v, recomputing P from the forward's log-sum-exp instead
+// of storing it ("Efficient attention: long context and sub-quadratic
+// variants", stanleyjacob.dev, section "Against the real libraries": the
+// production kernel line ships a recompute-based backward pass).
+//
+// For one (batch, query head) with S = scale q k^T (masked -inf) and
+// P = exp(S - lse) (lse from the forward), the chain rule gives
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D) with D_i = dO_i . O_i,
+//   dQ = scale dS K,  dK = scale dS^T Q,
+// and grouped KV heads sum the gradients of the query heads that read them.
+//
+// Three kernels, all on the caller's stream:
+//   attn_bwd_delta_kernel  D = rowsum(dO * O) in fp32 (the caller's workspace)
+//   attn_bwd_dq_kernel     one 128-row query tile per work item, walking its
+//                          visible K/V tiles: S = Q K^T and dP = dO V^T on the
+//                          tensor core, dS by the softmax warps, dQ += dS K
+//   attn_bwd_dkdv_kernel   one 128-key K/V tile per work item, walking the
+//                          visible query tiles of every query head of its KV
+//                          group: S^T = K Q^T, dP^T = V dO^T, P^T and dS^T by
+//                          the softmax warps, dV += P^T dO, dK += dS^T Q
+// so every accumulator stays in TMEM for a whole work item and nothing is
+// accumulated through global atomics.
+//
+// CTA organisation of both tcgen05 kernels (192 threads, one CTA per SM,
+// persistent): warps 0-3 elementwise (thread = TMEM lane = one row of the
+// work item's tile), warp 4 TMA loader, warp 5 tcgen05 issuer (one elected
+// lane issues).  All waits are bounded like the forward's.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace attn_sm100_bwd {
+using namespace attn_sm100;
+
+constexpr int kTile = 128;  // rows of every Q / dO / K / V tile
+constexpr int kBwdThreads = 192;
+constexpr int kBwdLoaderWarp = 4;
+constexpr int kBwdMmaWarp = 5;
+constexpr uint32_t kBwdTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+enum : int { kBMaskFull = 0, kBMaskCausal = 1, kBMaskWindow = 2 };
+enum : int { kBRoleLoader = 1, kBRoleMma = 2, kBRoleElem = 3, kBKernelDq = 0, kBKernelDkdv = 1 };
+
+struct BwdParams {
+  CUtensorMap tm_q;   // [B*Hq, N, d] bf16, box 64 x 128, 128-byte swizzle
+  CUtensorMap tm_k;   // [B*Hkv, N, d]
+  CUtensorMap tm_v;   // [B*Hkv, N, d]
+  CUtensorMap tm_do;  // [B*Hq, N, d]
+  const float* lse;   // [B*Hq, N] natural-log LSE from the forward
+  const float* delta; // [B*Hq, N] D = rowsum(dO * O)
+  __nv_bfloat16* dq;  // [B*Hq, N, d]
+  __nv_bfloat16* dk;  // [B*Hkv, N, d]
+  __nv_bfloat16* dv;  // [B*Hkv, N, d]
+  int* err;           // device error word (shared with the forward)
+  int B, Hq, Hkv, N, group;
+  int mask_kind, window;
+  float scale;        // softmax scale (dQ, dK are scaled by it)
+  float scale_log2;   // scale * log2(e)
+  int num_blk;        // ceil(N / 128)
+  int num_items;      // work items of the kernel being launched
+  unsigned long long timeout_ns;
+};
+
+// Visible key range [lo, hi] (tile indices) of query tile m, and visible query
+// tile range of key tile n (the transposed question), for the three masks.
+__device__ __forceinline__ void key_tiles_of_query_tile(const BwdParams& p, int m, int& lo, int& hi) {
+  const int r0 = m * kTile;
+  const int r1 = min(r0 + kTile - 1, p.N - 1);
+  if (p.mask_kind == kBMaskFull) {
+    lo = 0;
+    hi = p.num_blk - 1;
+  } else {
+    hi = r1 / kTile;
+    lo = (p.mask_kind == kBMaskWindow) ? max(0, r0 - p.window + 1) / kTile : 0;
+  }
+}
+__device__ __forceinline__ void query_tiles_of_key_tile(const BwdParams& p, int n, int& lo, int& hi) {
+  const int c0 = n * kTile;
+  const int c1 = min(c0 + kTile - 1, p.N - 1);
+  if (p.mask_kind == kBMaskFull) {
+    lo = 0;
+    hi = p.num_blk - 1;
+  } else {
+    lo = c0 / kTile;  // query i sees key j only if j <= i
+    // window: key j is seen by queries i with j <= i <= j + w - 1
+    hi = (p.mask_kind == kBMaskWindow) ? min(p.num_blk - 1, (c1 + p.window - 1) / kTile) : p.num_blk - 1;
+  }
+}
+// Is key j visible to query i (both absolute indices)?
+__device__ __forceinline__ bool key_visible(const BwdParams& p, int i, int j) {
+  if (i >= p.N || j >= p.N) return false;
+  if (p.mask_kind == kBMaskFull) return true;
+  if (j > i) return false;
+  return p.mask_kind != kBMaskWindow || j > i - p.window;
+}
+// Does the (query tile m, key tile n) block need element masks?
+__device__ __forceinline__ bool block_is_partial(const BwdParams& p, int m, int n) {
+  const int r0 = m * kTile, c0 = n * kTile;
+  bool partial = (c0 + kTile > p.N) || (r0 + kTile > p.N);
+  if (p.mask_kind != kBMaskFull) partial |= (c0 + kTile - 1 > r0);
+  if (p.mask_kind == kBMaskWindow) partial |= (c0 <= r0 + kTile - 1 - p.window);
+  return partial;
+}
+
+// Bounded mbarrier waits (a wait that gives up records `code` in the error
+// word and raises the CTA's abort flag; the roles then leave their loops).
+struct BwdWaiter {
+  uint64_t limit_ns;
+  volatile int* abort_flag;
+  int* err;
+  __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, int code) const {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        atomicCAS(err, 0, code);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+  __device__ __forceinline__ bool drain(uint32_t bar, uint32_t parity, int code) const {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+      if (global_timer_ns() - t0 > limit_ns) {
+        atomicCAS(err, 0, code);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+    return true;
+  }
+  // All 32 lanes wait; true only if every lane saw the phase.
+  __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, int code) const {
+    return __all_sync(0xffffffffu, wait(bar, parity, code));
+  }
+};
+
+__device__ __forceinline__ float bexp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// ------------------------------------------------------------------ delta
+// D[row] = sum_c dO[row, c] * O[row, c] in fp32 from bf16, one row per 16
+// threads (8 elements each, 16-byte loads), rows = B * Hq * N.
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __nv_bfloat16* __restrict__ out,
+                                                            const __nv_bfloat16* __restrict__ dout,
+                                                            float* __restrict__ delta, int64_t rows) {
+  constexpr int kThreadsPerRow = D / 8;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t row = t / kThreadsPerRow;
+  const int part = static_cast<int>(t % kThreadsPerRow);
+  float acc = 0.f;
+  if (row < rows) {
+    const uint4 a = *reinterpret_cast<const uint4*>(out + row * D + part * 8);
+    const uint4 b = *reinterpret_cast<const uint4*>(dout + row * D + part * 8);
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc = fmaf(__uint_as_float(av[i] << 16), __uint_as_float(bv[i] << 16), acc);
+      acc = fmaf(__uint_as_float(av[i] & 0xffff0000u), __uint_as_float(bv[i] & 0xffff0000u), acc);
+    }
+  }
+#pragma unroll
+  for (int o = kThreadsPerRow / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (row < rows && part == 0) delta[row] = acc;
+}
+
+// ------------------------------------------------------------------ layouts
+// dQ kernel: Q and dO tiles of the work item, then a ring of (K_j, V_j) stages.
+// dK/dV kernel: K and V tiles of the work item, then a ring of (Q_i, dO_i)
+// stages, plus the per-step log-sum-exp and D vectors of the query tile.
+template <int D>
+struct BwdSmem {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int kChunks = D / 64;                        // 128-byte column chunks
+  static constexpr uint32_t kChunkBytes = kTile * 128;          // 128 rows x 128 B
+  static constexpr uint32_t kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStages = (D == 128) ? 2 : 4;
+  static constexpr uint32_t kFixOff = 0;                        // two fixed tiles
+  static constexpr uint32_t kRingOff = 2 * kTileBytes;          // stages of two tiles
+  static constexpr uint32_t kVecOff = kRingOff + kStages * 2 * kTileBytes;  // 4 warps x (lse2, D) x 128 floats
+  static constexpr uint32_t kBarOff = kVecOff + 4 * 2 * kTile * 4;
+  static constexpr int kFixFull = 0;
+  static constexpr int kFixEmpty = 1;
+  static constexpr int kRingFull = 2;
+  static constexpr int kRingEmpty = kRingFull + kStages;
+  static constexpr int kSFull = kRingEmpty + kStages;
+  static constexpr int kPFull = kSFull + 1;
+  static constexpr int kAccDone = kPFull + 1;
+  static constexpr int kAccFree = kAccDone + 1;
+  static constexpr int kFin = kAccFree + 1;
+  static constexpr int kNumBars = kFin + 1;
+  static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr uint32_t kBytes = kMiscOff + 16;
+  static constexpr uint32_t kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
+  // TMEM columns: scores (or S^T), dP (or dP^T), then the accumulators.
+  static constexpr uint32_t kColS = 0, kColP = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
+};
+
+// Operand descriptors of a tile stored as 128 rows x D (K-major: the D axis
+// is the reduction axis) or read as the MN-major B operand of a TS MMA (the
+// 128 rows are the reduction axis).
+template <int D>
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr) {
+  return smem_desc_sw128(saddr, 16, 1024);
+}
+template <int D>
+__device__ __forceinline__ uint32_t kmajor_off(int kk) {
+  return ((kk >> 2) * BwdSmem<D>::kChunkBytes + (kk & 3) * 32) >> 4;
+}
+template <int D>
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t saddr) {
+  return smem_desc_sw128(saddr, BwdSmem<D>::kChunkBytes, 1024);
+}
+
+// Store one 128-column-or-less fp32 TMEM row segment (this thread's row) as
+// bf16 times `mul` to a global row; TMEM columns [col0, col0 + D).
+template <int D>
+__device__ __forceinline__ void store_acc_row(uint32_t tacc, float mul, __nv_bfloat16* dst_row, bool ok) {
+#pragma unroll 1
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t o[32];
+    tmem_load_32cols(tacc + cc * 32, o);
+    if (ok) {
+      uint32_t h[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) h[i] = bf16x2_rn(__uint_as_float(o[2 * i]) * mul, __uint_as_float(o[2 * i + 1]) * mul);
+      uint4* dst = reinterpret_cast<uint4*>(dst_row) + cc * 4;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) dst[v] = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ dQ kernel
+struct DqItem {
+  int b, hq, hkv, m, lo, hi;
+};
+__device__ __forceinline__ DqItem dq_item(const BwdParams& p, int i) {
+  DqItem it;
+  const int bh = i / p.num_blk;
+  it.m = p.num_blk - 1 - (i - bh * p.num_blk);  // longest query tile of a head first
+  it.b = bh / p.Hq;
+  it.hq = bh - it.b * p.Hq;
+  it.hkv = it.hq / p.group;
+  key_tiles_of_query_tile(p, it.m, it.lo, it.hi);
+  return it;
+}
+
+template <int D>
+__device__ __forceinline__ void dq_loader(const BwdParams& p, uint32_t sbase, const BwdWaiter& w) {
+  using L = BwdSmem<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  const uint64_t pol_kv = l2_policy_evict_last();
+  const uint64_t pol_q = l2_policy_evict_first();
+  uint32_t n = 0;         // ring loads issued
+  uint32_t fix_issued = 0;  // Q / dO tile pairs issued
+  int items = 0;
+  bool ok = true;
+  for (int i = blockIdx.x; ok && i < p.num_items; i += gridDim.x, ++items) {
+    const DqItem it = dq_item(p, i);
+    if (items > 0 && !w.wait(bar(L::kFixEmpty), (items - 1) & 1, (kBKernelDq << 12) | (kBRoleLoader << 8) | L::kFixEmpty)) {
+      ok = false;
+      break;
+    }
+    mbar_arrive_expect_tx(bar(L::kFixFull), 2 * L::kTileBytes);
+    ++fix_issued;
+    const int zq = it.b * p.Hq + it.hq;
+#pragma unroll
+    for (int c = 0; c < L::kChunks; ++c) {
+      tma_load_3d(sbase + L::kFixOff + c * L::kChunkBytes, &p.tm_q, bar(L::kFixFull), c * 64, it.m * kTile, zq, pol_q);
+      tma_load_3d(sbase + L::kFixOff + L::kTileBytes + c * L::kChunkBytes, &p.tm_do, bar(L::kFixFull), c * 64,
+                  it.m * kTile, zq, pol_q);
+    }
+    const int zk = it.b * p.Hkv + it.hkv;
+    for (int j = it.lo; j <= it.hi; ++j, ++n) {
+      const uint32_t slot = n % L::kStages;
+      if (n >= (uint32_t)L::kStages &&
+          !w.wait(bar(L::kRingEmpty + slot), ((n / L::kStages) - 1) & 1,
+                  (kBKernelDq << 12) | (kBRoleLoader << 8) | (L::kRingEmpty + slot))) {
+        ok = false;
+        break;
+      }
+      const uint32_t dst = sbase + L::kRingOff + slot * 2 * L::kTileBytes;
+      mbar_arrive_expect_tx(bar(L::kRingFull + slot), 2 * L::kTileBytes);
+#pragma unroll
+      for (int c = 0; c < L::kChunks; ++c) {
+        tma_load_3d(dst + c * L::kChunkBytes, &p.tm_k, bar(L::kRingFull + slot), c * 64, j * kTile, zk, pol_kv);
+        tma_load_3d(dst + L::kTileBytes + c * L::kChunkBytes, &p.tm_v, bar(L::kRingFull + slot), c * 64, j * kTile, zk,
+                    pol_kv);
+      }
+    }
+  }
+  // Drain: every copy this thread started must land before the CTA exits.
+  for (uint32_t s = 0; s < (uint32_t)L::kStages; ++s) {
+    if (n > s) {
+      const uint32_t last = s + ((n - 1 - s) / L::kStages) * L::kStages;
+      w.drain(bar(L::kRingFull + s), (last / L::kStages) & 1, (kBKernelDq << 12) | (kBRoleLoader << 8) | (L::kRingFull + s));
+    }
+  }
+  if (fix_issued > 0)
+    w.drain(bar(L::kFixFull), (fix_issued - 1) & 1, (kBKernelDq << 12) | (kBRoleLoader << 8) | L::kFixFull);
+}
+
+template <int D>
+__device__ __forceinline__ void dq_mma(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w) {
+  using L = BwdSmem<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  constexpr uint32_t idesc_ss = idesc_bf16_f32(kTile, kTile, false);
+  constexpr uint32_t idesc_ts = idesc_bf16_f32(kTile, D, true);
+  const uint32_t t_s = tmem + L::kColS, t_p = tmem + L::kColP, t_acc = tmem + L::kColAcc0;
+  const uint64_t q_desc = kmajor_desc<D>(sbase + L::kFixOff);
+  const uint64_t do_desc = kmajor_desc<D>(sbase + L::kFixOff + L::kTileBytes);
+  const int code = (kBKernelDq << 12) | (kBRoleMma << 8);
+  uint32_t n = 0, ds_cnt = 0;
+  int items = 0;
+  bool ok = true;
+  for (int i = blockIdx.x; ok && i < p.num_items; i += gridDim.x, ++items) {
+    const DqItem it = dq_item(p, i);
+    if (!w.wait_warp(bar(L::kFixFull), items & 1, code | L::kFixFull)) break;
+    tc_fence_after_sync();
+    for (int j = it.lo; j <= it.hi; ++j, ++n) {
+      const uint32_t slot = n % L::kStages;
+      const uint32_t kaddr = sbase + L::kRingOff + slot * 2 * L::kTileBytes;
+      if (!w.wait_warp(bar(L::kRingFull + slot), (n / L::kStages) & 1, code | (L::kRingFull + slot))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      const uint64_t k_desc = kmajor_desc<D>(kaddr), v_desc = kmajor_desc<D>(kaddr + L::kTileBytes);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = kmajor_off<D>(kk);
+        mma_bf16_ss_elect(t_s, q_desc + off, k_desc + off, idesc_ss, kk > 0 ? 1u : 0u);   // S = Q K^T
+        mma_bf16_ss_elect(t_p, do_desc + off, v_desc + off, idesc_ss, kk > 0 ? 1u : 0u);  // dP = dO V^T
+      }
+      tc_commit_elect(bar(L::kSFull));
+      if (j == it.hi) tc_commit_elect(bar(L::kFixEmpty));  // Q, dO read
+      if (!w.wait_warp(bar(L::kPFull), ds_cnt & 1, code | L::kPFull)) {
+        ok = false;
+        break;
+      }
+      ++ds_cnt;
+      if (j == it.lo && items > 0 && !w.wait_warp(bar(L::kAccFree), (items - 1) & 1, code | L::kAccFree)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      const uint64_t kb_desc = mnmajor_desc<D>(kaddr);
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk)  // dQ += dS K (dS in TMEM over the S columns)
+        mma_bf16_ts_elect(t_acc, t_s + kk * 8, kb_desc + ((kk * 2048) >> 4), idesc_ts, (kk > 0 || j > it.lo) ? 1u : 0u);
+      tc_commit_elect(bar(L::kRingEmpty + slot));
+    }
+    if (!ok) break;
+    tc_commit_elect(bar(L::kAccDone));
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void dq_elem(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w,
+                                        int warp, int lane) {
+  using L = BwdSmem<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  const int r = warp * 32 + lane;  // row of the query tile = TMEM lane
+  const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t t_s = tmem + lane_bits + L::kColS, t_p = tmem + lane_bits + L::kColP;
+  const uint32_t t_acc = tmem + lane_bits + L::kColAcc0;
+  const float c2 = p.scale_log2;
+  const int code = (kBKernelDq << 12) | (kBRoleElem << 8);
+  uint32_t s_cnt = 0;
+  int items = 0;
+  for (int i = blockIdx.x; i < p.num_items; i += gridDim.x, ++items) {
+    const DqItem it = dq_item(p, i);
+    const int row = it.m * kTile + r;
+    const bool row_ok = row < p.N;
+    const size_t bhrow = (static_cast<size_t>(it.b) * p.Hq + it.hq) * p.N + (row_ok ? row : 0);
+    const float lse2 = row_ok ? p.lse[bhrow] * kLog2e : 0.f;
+    const float dlt = row_ok ? p.delta[bhrow] : 0.f;
+    bool ok = true;
+    for (int j = it.lo; j <= it.hi; ++j) {
+      if (!w.wait_warp(bar(L::kSFull), s_cnt & 1, code | L::kSFull)) {
+        ok = false;
+        break;
+      }
+      ++s_cnt;
+      tc_fence_after_sync();
+      const bool partial = block_is_partial(p, it.m, j);
+#pragma unroll
+      for (int chunk = 0; chunk < 4; ++chunk) {
+        uint32_t sv[32], pv[32];
+        tmem_load_32cols(t_s + chunk * 32, sv);
+        tmem_load_32cols(t_p + chunk * 32, pv);
+        uint32_t packed[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float ds[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float pr = bexp2(__uint_as_float(sv[e + h]) * c2 - lse2);
+            if (partial && !key_visible(p, row, j * kTile + chunk * 32 + e + h)) pr = 0.f;
+            ds[h] = pr * (__uint_as_float(pv[e + h]) - dlt);
+          }
+          packed[e >> 1] = bf16x2_rn(ds[0], ds[1]);
+        }
+        tmem_store_16cols(t_s + chunk * 16, packed);  // dS over the first half of the S columns
+      }
+      tmem_store_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::kPFull));
+    }
+    if (!ok) break;
+    if (!w.wait_warp(bar(L::kAccDone), items & 1, code | L::kAccDone)) break;
+    tc_fence_after_sync();
+    store_acc_row<D>(t_acc, p.scale, p.dq + bhrow * D, row_ok);
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(L::kAccFree));
+  }
+  tmem_store_wait();
+}
+
+// ------------------------------------------------------------------ dK/dV kernel
+struct DkvItem {
+  int b, hkv, n, qlo, qhi, steps;  // steps = group * (qhi - qlo + 1)
+};
+__device__ __forceinline__ DkvItem dkv_item(const BwdParams& p, int i) {
+  DkvItem it;
+  const int bk = i / p.num_blk;
+  it.n = i - bk * p.num_blk;  // under a causal mask the first key tiles see the most queries
+  it.b = bk / p.Hkv;
+  it.hkv = bk - it.b * p.Hkv;
+  query_tiles_of_key_tile(p, it.n, it.qlo, it.qhi);
+  it.steps = p.group * (it.qhi - it.qlo + 1);
+  return it;
+}
+// Step s of an item: query head hkv * group + s / (qhi - qlo + 1), query tile qlo + s % (...).
+__device__ __forceinline__ void dkv_step(const BwdParams& p, const DkvItem& it, int s, int& hq, int& m) {
+  const int per_head = it.qhi - it.qlo + 1;
+  const int h = s / per_head;
+  hq = it.hkv * p.group + h;
+  m = it.qlo + (s - h * per_head);
+}
+
+template <int D>
+__device__ __forceinline__ void dkv_loader(const BwdParams& p, uint32_t sbase, const BwdWaiter& w) {
+  using L = BwdSmem<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  const uint64_t pol_kv = l2_policy_evict_first();
+  const uint64_t pol_q = l2_policy_evict_last();
+  const int code = (kBKernelDkdv << 12) | (kBRoleLoader << 8);
+  uint32_t n = 0;
+  uint32_t fix_issued = 0;  // K / V tile pairs issued
+  int items = 0;
+  bool ok = true;
+  for (int i = blockIdx.x; ok && i < p.num_items; i += gridDim.x, ++items) {
+    const DkvItem it = dkv_item(p, i);
+    if (items > 0 && !w.wait(bar(L::kFixEmpty), (items - 1) & 1, code | L::kFixEmpty)) {
+      ok = false;
+      break;
+    }
+    mbar_arrive_expect_tx(bar(L::kFixFull), 2 * L::kTileBytes);
+    ++fix_issued;
+    const int zk = it.b * p.Hkv + it.hkv;
+#pragma unroll
+    for (int c = 0; c < L::kChunks; ++c) {
+      tma_load_3d(sbase + L::kFixOff + c * L::kChunkBytes, &p.tm_k, bar(L::kFixFull), c * 64, it.n * kTile, zk, pol_kv);
+      tma_load_3d(sbase + L::kFixOff + L::kTileBytes + c * L::kChunkBytes, &p.tm_v, bar(L::kFixFull), c * 64,
+                  it.n * kTile, zk, pol_kv);
+    }
+    for (int s = 0; s < it.steps; ++s, ++n) {
+      int hq, m;
+      dkv_step(p, it, s, hq, m);
+      const uint32_t slot = n % L::kStages;
+      if (n >= (uint32_t)L::kStages &&
+          !w.wait(bar(L::kRingEmpty + slot), ((n / L::kStages) - 1) & 1, code | (L::kRingEmpty + slot))) {
+        ok = false;
+        break;
+      }
+      const uint32_t dst = sbase + L::kRingOff + slot * 2 * L::kTileBytes;
+      const int zq = it.b * p.Hq + hq;
+      mbar_arrive_expect_tx(bar(L::kRingFull + slot), 2 * L::kTileBytes);
+#pragma unroll
+      for (int c = 0; c < L::kChunks; ++c) {
+        tma_load_3d(dst + c * L::kChunkBytes, &p.tm_q, bar(L::kRingFull + slot), c * 64, m * kTile, zq, pol_q);
+        tma_load_3d(dst + L::kTileBytes + c * L::kChunkBytes, &p.tm_do, bar(L::kRingFull + slot), c * 64, m * kTile, zq,
+                    pol_q);
+      }
+    }
+  }
+  for (uint32_t s = 0; s < (uint32_t)L::kStages; ++s) {
+    if (n > s) {
+      const uint32_t last = s + ((n - 1 - s) / L::kStages) * L::kStages;
+      w.drain(bar(L::kRingFull + s), (last / L::kStages) & 1, code | (L::kRingFull + s));
+    }
+  }
+  if (fix_issued > 0) w.drain(bar(L::kFixFull), (fix_issued - 1) & 1, code | L::kFixFull);
+}
+
+template <int D>
+__device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w) {
+  using L = BwdSmem<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  constexpr uint32_t idesc_ss = idesc_bf16_f32(kTile, kTile, false);
+  constexpr uint32_t idesc_ts = idesc_bf16_f32(kTile, D, true);
+  const uint32_t t_s = tmem + L::kColS, t_p = tmem + L::kColP;
+  const uint32_t t_dv = tmem + L::kColAcc0, t_dk = tmem + L::kColAcc1;
+  const uint64_t k_desc = kmajor_desc<D>(sbase + L::kFixOff);
+  const uint64_t v_desc = kmajor_desc<D>(sbase + L::kFixOff + L::kTileBytes);
+  const int code = (kBKernelDkdv << 12) | (kBRoleMma << 8);
+  uint32_t n = 0, p_cnt = 0;
+  int items = 0;
+  bool ok = true;
+  for (int i = blockIdx.x; ok && i < p.num_items; i += gridDim.x, ++items) {
+    const DkvItem it = dkv_item(p, i);
+    if (!w.wait_warp(bar(L::kFixFull), items & 1, code | L::kFixFull)) break;
+    tc_fence_after_sync();
+    for (int s = 0; s < it.steps; ++s, ++n) {
+      const uint32_t slot = n % L::kStages;
+      const uint32_t qaddr = sbase + L::kRingOff + slot * 2 * L::kTileBytes;
+      if (!w.wait_warp(bar(L::kRingFull + slot), (n / L::kStages) & 1, code | (L::kRingFull + slot))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      const uint64_t q_desc = kmajor_desc<D>(qaddr), do_desc = kmajor_desc<D>(qaddr + L::kTileBytes);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = kmajor_off<D>(kk);
+        mma_bf16_ss_elect(t_s, k_desc + off, q_desc + off, idesc_ss, kk > 0 ? 1u : 0u);   // S^T = K Q^T
+        mma_bf16_ss_elect(t_p, v_desc + off, do_desc + off, idesc_ss, kk > 0 ? 1u : 0u);  // dP^T = V dO^T
+      }
+      tc_commit_elect(bar(L::kSFull));
+      if (s == it.steps - 1) tc_commit_elect(bar(L::kFixEmpty));  // K, V read
+      if (!w.wait_warp(bar(L::kPFull), p_cnt & 1, code | L::kPFull)) {
+        ok = false;
+        break;
+      }
+      ++p_cnt;
+      if (s == 0 && items > 0 && !w.wait_warp(bar(L::kAccFree), (items - 1) & 1, code | L::kAccFree)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      const uint64_t dob_desc = mnmajor_desc<D>(qaddr + L::kTileBytes), qb_desc = mnmajor_desc<D>(qaddr);
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk) {
+        const uint32_t acc = (kk > 0 || s > 0) ? 1u : 0u;
+        mma_bf16_ts_elect(t_dv, t_s + kk * 8, dob_desc + ((kk * 2048) >> 4), idesc_ts, acc);  // dV += P^T dO
+        mma_bf16_ts_elect(t_dk, t_p + kk * 8, qb_desc + ((kk * 2048) >> 4), idesc_ts, acc);   // dK += dS^T Q
+      }
+      tc_commit_elect(bar(L::kRingEmpty + slot));
+    }
+    if (!ok) break;
+    tc_commit_elect(bar(L::kAccDone));
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w,
+                                         int warp, int lane) {
+  using L = BwdSmem<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  const int r = warp * 32 + lane;  // key row of the tile = TMEM lane
+  const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t t_s = tmem + lane_bits + L::kColS, t_p = tmem + lane_bits + L::kColP;
+  const uint32_t t_dv = tmem + lane_bits + L::kColAcc0, t_dk = tmem + lane_bits + L::kColAcc1;
+  // This warp's copy of the step's log2-scaled LSE and D of the 128 query rows.
+  float* s_lse = reinterpret_cast<float*>(__cvta_shared_to_generic(sbase + L::kVecOff)) + warp * 2 * kTile;
+  float* s_dlt = s_lse + kTile;
+  const float c2 = p.scale_log2;
+  const int code = (kBKernelDkdv << 12) | (kBRoleElem << 8);
+  uint32_t s_cnt = 0;
+  int items = 0;
+  for (int i = blockIdx.x; i < p.num_items; i += gridDim.x, ++items) {
+    const DkvItem it = dkv_item(p, i);
+    const int key = it.n * kTile + r;
+    bool ok = true;
+    for (int s = 0; s < it.steps; ++s) {
+      int hq, m;
+      dkv_step(p, it, s, hq, m);
+      {
+        const size_t bhq = (static_cast<size_t>(it.b) * p.Hq + hq) * p.N;
+        __syncwarp();  // the previous step's reads of this warp's copy are done
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int c = lane + 32 * t, q = m * kTile + c;
+          s_lse[c] = (q < p.N) ? p.lse[bhq + q] * kLog2e : 0.f;
+          s_dlt[c] = (q < p.N) ? p.delta[bhq + q] : 0.f;
+        }
+        __syncwarp();
+      }
+      if (!w.wait_warp(bar(L::kSFull), s_cnt & 1, code | L::kSFull)) {
+        ok = false;
+        break;
+      }
+      ++s_cnt;
+      tc_fence_after_sync();
+      const bool partial = block_is_partial(p, m, it.n);
+#pragma unroll
+      for (int chunk = 0; chunk < 4; ++chunk) {
+        uint32_t sv[32], pv[32];
+        tmem_load_32cols(t_s + chunk * 32, sv);
+        tmem_load_32cols(t_p + chunk * 32, pv);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pr[2], ds[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int c = chunk * 32 + e + h;  // query column within the tile
+            float x = bexp2(__uint_as_float(sv[e + h]) * c2 - s_lse[c]);
+            if (partial && !key_visible(p, m * kTile + c, key)) x = 0.f;
+            pr[h] = x;
+            ds[h] = x * (__uint_as_float(pv[e + h]) - s_dlt[c]);
+          }
+          pk[e >> 1] = bf16x2_rn(pr[0], pr[1]);
+          dk[e >> 1] = bf16x2_rn(ds[0], ds[1]);
+        }
+        tmem_store_16cols(t_s + chunk * 16, pk);  // P^T over the first half of the S^T columns
+        tmem_store_16cols(t_p + chunk * 16, dk);  // dS^T over the first half of the dP^T columns
+      }
+      tmem_store_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::kPFull));
+    }
+    if (!ok) break;
+    if (!w.wait_warp(bar(L::kAccDone), items & 1, code | L::kAccDone)) break;
+    tc_fence_after_sync();
+    const bool key_ok = key < p.N;
+    const size_t krow = (static_cast<size_t>(it.b) * p.Hkv + it.hkv) * p.N + (key_ok ? key : 0);
+    store_acc_row<D>(t_dv, 1.f, p.dv + krow * D, key_ok);
+    store_acc_row<D>(t_dk, p.scale, p.dk + krow * D, key_ok);
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(L::kAccFree));
+  }
+  tmem_store_wait();
+}
+
+// ------------------------------------------------------------------ entry
+template <int D, int KIND>
+__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_constant__ BwdParams p) {
+  using L = BwdSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  if (threadIdx.x == 0) {
+    auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+    mbar_init(bar(L::kFixFull), 1);
+    mbar_init(bar(L::kFixEmpty), 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar(L::kRingFull + s), 1);
+      mbar_init(bar(L::kRingEmpty + s), 1);
+    }
+    mbar_init(bar(L::kSFull), 1);
+    mbar_init(bar(L::kPFull), 4);    // one arrival per elementwise warp
+    mbar_init(bar(L::kAccDone), 1);
+    mbar_init(bar(L::kAccFree), 4);  // one arrival per elementwise warp
+    mbar_init(bar(L::kFin), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), kBwdTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const BwdWaiter w{p.timeout_ns, abort_flag, p.err};
+  if (warp < 4) {
+    if (KIND == kBKernelDq) dq_elem<D>(p, sbase, tmem, w, warp, lane);
+    else dkv_elem<D>(p, sbase, tmem, w, warp, lane);
+  } else if (warp == kBwdLoaderWarp) {
+    if (lane == 0) {
+      if (KIND == kBKernelDq) dq_loader<D>(p, sbase, w);
+      else dkv_loader<D>(p, sbase, w);
+    }
+    __syncwarp();
+  } else if (warp == kBwdMmaWarp) {
+    if (KIND == kBKernelDq) dq_mma<D>(p, sbase, tmem, w);
+    else dkv_mma<D>(p, sbase, tmem, w);
+    // Every MMA this warp issued must complete before TMEM is freed.
+    tc_commit_elect(sbase + L::kBarOff + 8u * L::kFin);
+    w.drain(sbase + L::kBarOff + 8u * L::kFin, 0, (KIND << 12) | (kBRoleMma << 8) | L::kFin);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kBwdTmemCols);
+  }
+}
+
+}  // namespace attn_sm100_bwd

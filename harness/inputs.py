@@ -103,3 +103,12 @@ def sample_rows(N: int, window: Optional[int], seed: int, count: int = 256) -> n
     rest = np.setdiff1d(np.arange(N, dtype=np.int64), np.fromiter(fixed, dtype=np.int64))
     extra = rng.choice(rest, size=count - len(fixed), replace=False)
     return np.sort(np.concatenate([np.fromiter(fixed, dtype=np.int64), extra]))
+
+
+def make_dout(B, Hq, N, d, seed, device="cpu", dtype=torch.bfloat16):
+    """Upstream gradient dO [B,Hq,N,d] for the backward: fp32 N(0,1) from a
+    generator seeded with ``seed + 7919`` (so it differs from q for the same
+    seed), rounded to bf16."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed) + 7919)
+    return torch.randn((B, Hq, N, d), generator=gen, device=device, dtype=torch.float32).to(dtype)

@@ -1,5 +1,5 @@
 /*
- * Exact attention forward for NVIDIA B200 (sm_100a): C ABI.
+ * Exact attention forward and backward for NVIDIA B200 (sm_100a): C ABI.
  *
  * Computes, for every batch b, query head h and query row i,
  *
@@ -30,6 +30,7 @@
 #ifndef ATTN_B200_ATTN_H_
 #define ATTN_B200_ATTN_H_
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
@@ -111,6 +112,50 @@ int attn_debug_error(cudaStream_t stream, int* device_code);
    helper for tests and tools; returns -1 on invalid sizes). */
 int64_t attn_fwd_num_work_items(int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
                                 int mask_kind, int64_t window);
+
+/*
+ * attn_bwd: enqueue the backward pass on `stream`: the gradients of sum(dout * out)
+ * with respect to q, k and v for the forward above (same masks, head map and scale).
+ * With S = scale q k^T (masked entries -inf) and P = exp(S - lse) per query row, the
+ * chain rule gives dV = P^T dO, dP = dO V^T, dS = P (dP - D) with D_i = dO_i . O_i,
+ * dQ = scale dS K and dK = scale dS^T Q; a KV head's dK, dV sum over the query heads
+ * that read it. The pages name a recompute-based backward pass as part of the
+ * production kernel line ("Efficient attention: long context and sub-quadratic
+ * variants", stanleyjacob.dev, section "Against the real libraries"); P is recomputed
+ * from lse, never stored.
+ *
+ *   q, k, v    as attn_fwd (bf16, contiguous, 16-byte aligned)
+ *   out, lse   attn_fwd's outputs for these q, k, v, scale and mask (read only)
+ *   dout       device pointer, bf16, [B, Hq, N, d], contiguous, 16-byte aligned
+ *   dq         device pointer, bf16, [B, Hq,  N, d], 16-byte aligned; fully overwritten
+ *   dk, dv     device pointers, bf16, [B, Hkv, N, d], 16-byte aligned; fully overwritten
+ *   workspace  device pointer, 4-byte aligned, at least attn_bwd_workspace_bytes(B, Hq, N)
+ *              bytes, owned by the caller; holds D (fp32 [B, Hq, N]) between the kernels
+ *              of one call, so it must not be reused until the stream has passed the call
+ *   B, Hq, Hkv, N, d, scale, mask_kind, window, stream: as attn_fwd
+ *
+ * The library allocates nothing. Outputs and the workspace must not overlap each other
+ * or the inputs (ATTN_ERR_INVALID_ARG). Errors and bounded waits as attn_fwd; a wait
+ * that gives up leaves a code that attn_bwd_debug_error returns as ATTN_ERR_TIMEOUT.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+             int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
+             float scale, int mask_kind, int64_t window, cudaStream_t stream);
+
+/* attn_bwd with options (wait bound and CTA count as for attn_fwd_ex; inject_stall
+   is ignored); opts may be NULL. */
+int attn_bwd_ex(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
+                float scale, int mask_kind, int64_t window, cudaStream_t stream,
+                const attn_fwd_options* opts);
+
+/* Workspace bytes attn_bwd needs (4 * B * Hq * N); 0 for invalid sizes. */
+size_t attn_bwd_workspace_bytes(int64_t B, int64_t Hq, int64_t N);
+
+/* attn_debug_error for the backward kernels' error word (same contract). */
+int attn_bwd_debug_error(cudaStream_t stream, int* device_code);
 
 #ifdef __cplusplus
 }

@@ -21,7 +21,7 @@ def lib():
 def declared_functions():
     text = open(os.path.join(ROOT, "include", "attn.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:int|int64_t|const char\*)\s+(attn_\w+)\s*\(", text, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:int|int64_t|size_t|const char\*)\s+(attn_\w+)\s*\(", text, flags=re.M)))
 
 
 def test_header_declares_expected_entry_points():
@@ -97,3 +97,41 @@ def test_python_binding_validates_without_launching():
     with pytest.raises((TypeError, ValueError)):
         A.fwd(torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16), torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16),
               torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16))
+
+
+# ------------------------------------------------------------------ backward
+DO, DQ, DK, DV, WS = (0x10000000000 * (i + 6) for i in range(5))
+
+
+def call_bwd(lib, q=Q, k=K, v=V, o=O, l=L, do=DO, dq=DQ, dk=DK, dv=DV, ws=WS, ws_bytes=None, B=1, Hq=2, Hkv=2,
+             N=256, d=64, scale=0.125, mask=1, window=0):
+    if ws_bytes is None:
+        ws_bytes = 4 * B * Hq * N
+    return lib.attn_bwd(q, k, v, o, l, do, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, N, d, scale, mask, window, None)
+
+
+def test_backward_workspace_bytes(lib):
+    assert lib.attn_bwd_workspace_bytes(2, 32, 8192) == 4 * 2 * 32 * 8192
+    assert lib.attn_bwd_workspace_bytes(0, 1, 1) == 0 and lib.attn_bwd_workspace_bytes(1, 1, -1) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(do=None), 1), (dict(dq=None), 1), (dict(dk=None), 1), (dict(dv=None), 1), (dict(ws=None), 1),
+    (dict(o=None), 1), (dict(l=None), 1),
+    (dict(ws_bytes=4 * 2 * 256 - 4), 1), (dict(B=0), 1), (dict(Hq=6, Hkv=4), 1), (dict(mask=7), 1),
+    (dict(mask=2, window=0), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1),
+    (dict(d=32), 2), (dict(d=256), 2),
+    (dict(do=DO + 8), 3), (dict(dq=DQ + 8), 3), (dict(dk=DK + 4), 3), (dict(dv=DV + 2), 3), (dict(ws=WS + 2), 3),
+    (dict(dq=Q), 1), (dict(dk=V + 64), 1), (dict(dv=DO), 1), (dict(ws=L), 1), (dict(dk=DQ + 128), 1),
+    (dict(ws=DV + 256), 1),
+])
+def test_backward_invalid_arguments_rejected_before_launch(lib, kw, status):
+    assert call_bwd(lib, **kw) == status
+
+
+def test_backward_valid_arguments_reach_the_device_check(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    assert call_bwd(lib) == 4
+    assert call_bwd(lib, d=128, mask=2, window=10 ** 9) == 4
