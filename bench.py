@@ -7,7 +7,10 @@ visible (query, key) pair.  Inputs (384 MiB of q, k, v) are larger than the
 126 MB L2, so no flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload dense|gqa|swa|long|tiny] [--no-cpu-baseline]
+                  [--workload dense|gqa|swa|long|tiny] [--no-cpu-baseline] [--pass fwd|bwd]
+
+``--pass bwd`` times the backward pass instead (one GPU; 10*d FLOPs per visible
+pair, the five products of the gradient).
 
 With --gpus N > 1 the script runs under torchrun, one rank per GPU; every rank
 runs its own shard of the global batch (weak scaling, no data-path collective)
@@ -333,6 +336,91 @@ def run_ours(args, w):
         dist.destroy_process_group()
 
 
+BWD_METRIC = "attention bwd TFLOP/s (bf16, 10*d FLOPs per visible pair) and % of B200 dense peak"
+
+
+def bwd_cpu_baseline(w, q, k, v, do, target_s=15.0):
+    """The fp64 backward oracle on host cores for one query head (with its KV
+    head) over a prefix of the sequence short enough to finish in seconds."""
+    import oracle.attention_bwd_fp64 as G
+    from oracle import attention_fp64 as F
+    n = min(w.N, 2048)
+    while True:
+        qs = q[:1, :1, :n].float().numpy()
+        ks = k[:1, :1, :n].float().numpy()
+        vs = v[:1, :1, :n].float().numpy()
+        ds = do[:1, :1, :n].float().numpy()
+        t0 = time.perf_counter()
+        G.attention_bwd(qs, ks, vs, ds, w.scale, F.MASK_CAUSAL if w.mask == "causal" else
+                        (F.MASK_FULL if w.mask == "full" else F.MASK_SLIDING_WINDOW), w.window)
+        dt = time.perf_counter() - t0
+        if dt > target_s / 8 or n >= min(w.N, 8192):
+            break
+        n = min(w.N, 8192, n * 2)
+    flops = 10 * w.d * visible_pairs(n, w.mask, w.window)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"one query head and its KV head, first {n} positions of the {w.name} workload "
+                      f"(fp64 NumPy, scores materialised), {dt:.1f} s"}
+
+
+def run_backward(args, w):
+    """Backward pass on one GPU: each step is one attn_bwd call (D, dQ and
+    dK/dV kernels) on the forward's out and lse and a seeded dO."""
+    from harness.inputs import make_dout
+    from exact_io_aware_72_b200 import bwd, fwd
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, device=device, sharp=w.sharp)
+    do = make_dout(w.B, w.Hq, w.N, w.d, w.seed, device=device)
+    out, lse = fwd(q, k, v, scale=w.scale, mask=w.mask, window=w.window)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(w.B * w.Hq * w.N, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        bwd(q, k, v, out, lse, do, scale=w.scale, mask=w.mask, window=w.window, dq=dq, dk=dk, dv=dv,
+            workspace=ws, stream=stream)
+
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    clocks.mark(0)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    evs[0].record(stream)
+    for i in range(args.steps):
+        step()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize(device)
+    clocks.mark(1)
+    per_launch_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    total_ms = evs[0].elapsed_time(evs[-1])
+    clk = clocks.stop()
+    flops = 10 * w.B * w.Hq * w.d * visible_pairs(w.N, w.mask, w.window)
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (statistics.mean(per_launch_ms) / 1e3) / 1e12
+    line = {
+        "metric": BWD_METRIC, "pass": "bwd", "value": flops * args.steps / (total_ms / 1e3) / 1e12,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "mask": w.mask,
+                   "window": w.window, "sharp_rows": w.sharp, "l2": "inputs larger than L2 (no flush)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak))},
+        "gpu_launches": 3 * args.steps,
+        "launch_ms": {"median": statistics.median(per_launch_ms), "best": min(per_launch_ms)},
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = bwd_cpu_baseline(w, q.cpu(), k.cpu(), v.cpu(), do.cpu(), args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -346,6 +434,8 @@ def main():
                     help="B,Hq,Hkv,N,d: run this shape instead of a named workload (profiling sweeps)")
     ap.add_argument("--mask", choices=["full", "causal", "sliding_window"], default=None)
     ap.add_argument("--window", type=int, default=None)
+    ap.add_argument("--pass", dest="which", choices=["fwd", "bwd"], default="fwd",
+                    help="bwd: time the backward pass (one GPU) instead of the forward")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -358,6 +448,8 @@ def main():
                     window=args.window if mask == "sliding_window" else None, sharp=False)
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.which == "bwd":
+        run_backward(args, w)
     else:
         run_ours(args, w)
 

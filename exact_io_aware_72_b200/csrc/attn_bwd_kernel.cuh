@@ -92,13 +92,6 @@ __device__ __forceinline__ void query_tiles_of_key_tile(const BwdParams& p, int 
     hi = (p.mask_kind == kBMaskWindow) ? min(p.num_blk - 1, (c1 + p.window - 1) / kTile) : p.num_blk - 1;
   }
 }
-// Is key j visible to query i (both absolute indices)?
-__device__ __forceinline__ bool key_visible(const BwdParams& p, int i, int j) {
-  if (i >= p.N || j >= p.N) return false;
-  if (p.mask_kind == kBMaskFull) return true;
-  if (j > i) return false;
-  return p.mask_kind != kBMaskWindow || j > i - p.window;
-}
 // Does the (query tile m, key tile n) block need element masks?
 __device__ __forceinline__ bool block_is_partial(const BwdParams& p, int m, int n) {
   const int r0 = m * kTile, c0 = n * kTile;
@@ -143,6 +136,25 @@ struct BwdWaiter {
     return __all_sync(0xffffffffu, wait(bar, parity, code));
   }
 };
+
+// Two 32-column TMEM loads (32x32b shape: thread = lane, consecutive registers
+// = consecutive columns) completed by one wait.
+__device__ __forceinline__ void tmem_load_2x32cols(uint32_t ta, uint32_t tb, uint32_t (&a)[32], uint32_t (&b)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]), "=r"(a[8]),
+        "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]), "=r"(a[16]),
+        "=r"(a[17]), "=r"(a[18]), "=r"(a[19]), "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]), "=r"(a[24]),
+        "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31]), "=r"(b[0]),
+        "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]), "=r"(b[8]), "=r"(b[9]),
+        "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15]), "=r"(b[16]), "=r"(b[17]),
+        "=r"(b[18]), "=r"(b[19]), "=r"(b[20]), "=r"(b[21]), "=r"(b[22]), "=r"(b[23]), "=r"(b[24]), "=r"(b[25]),
+        "=r"(b[26]), "=r"(b[27]), "=r"(b[28]), "=r"(b[29]), "=r"(b[30]), "=r"(b[31])
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
 
 __device__ __forceinline__ float bexp2(float x) {
   float y;
@@ -403,25 +415,38 @@ __device__ __forceinline__ void dq_elem(const BwdParams& p, uint32_t sbase, uint
       ++s_cnt;
       tc_fence_after_sync();
       const bool partial = block_is_partial(p, it.m, j);
+      // Visible key columns of this row in the tile: lo_c <= c <= hi_c (only
+      // applied on partial tiles, where the masked scores become -inf).
+      const int j0 = j * kTile;
+      const int hi_c = row_ok ? min(p.N - 1, p.mask_kind == kBMaskFull ? p.N - 1 : row) - j0 : -1;
+      const int lo_c = (p.mask_kind == kBMaskWindow) ? row - p.window + 1 - j0 : 0;
+      // All loads before any store: dS (bf16, 64 columns) is kept in registers
+      // and written over the first half of the S columns at the end.
+      uint32_t packed[4][16];
 #pragma unroll
       for (int chunk = 0; chunk < 4; ++chunk) {
         uint32_t sv[32], pv[32];
-        tmem_load_32cols(t_s + chunk * 32, sv);
-        tmem_load_32cols(t_p + chunk * 32, pv);
-        uint32_t packed[16];
+        tmem_load_2x32cols(t_s + chunk * 32, t_p + chunk * 32, sv, pv);
+        if (partial) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int c = chunk * 32 + e;
+            if (c > hi_c || c < lo_c) sv[e] = 0xff800000u;  // -inf
+          }
+        }
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           float ds[2];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            float pr = bexp2(__uint_as_float(sv[e + h]) * c2 - lse2);
-            if (partial && !key_visible(p, row, j * kTile + chunk * 32 + e + h)) pr = 0.f;
+            const float pr = bexp2(__uint_as_float(sv[e + h]) * c2 - lse2);
             ds[h] = pr * (__uint_as_float(pv[e + h]) - dlt);
           }
-          packed[e >> 1] = bf16x2_rn(ds[0], ds[1]);
+          packed[chunk][e >> 1] = bf16x2_rn(ds[0], ds[1]);
         }
-        tmem_store_16cols(t_s + chunk * 16, packed);  // dS over the first half of the S columns
       }
+#pragma unroll
+      for (int chunk = 0; chunk < 4; ++chunk) tmem_store_16cols(t_s + chunk * 16, packed[chunk]);
       tmem_store_wait();
       tc_fence_before_sync();
       __syncwarp();
@@ -615,28 +640,45 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
       ++s_cnt;
       tc_fence_after_sync();
       const bool partial = block_is_partial(p, m, it.n);
+      // Query columns that see this key: lo_c <= c <= hi_c (only applied on
+      // partial tiles, where the masked scores become -inf).
+      const int q0 = m * kTile;
+      const int hi_c = (key < p.N)
+                           ? min(p.N - 1, p.mask_kind == kBMaskWindow ? key + p.window - 1 : p.N - 1) - q0
+                           : -1;
+      const int lo_c = (p.mask_kind == kBMaskFull) ? 0 : key - q0;
+      // All loads before any store: P^T and dS^T (bf16, 64 columns each) are
+      // kept in registers and written over the first halves at the end.
+      uint32_t pk[4][16], dk[4][16];
 #pragma unroll
       for (int chunk = 0; chunk < 4; ++chunk) {
         uint32_t sv[32], pv[32];
-        tmem_load_32cols(t_s + chunk * 32, sv);
-        tmem_load_32cols(t_p + chunk * 32, pv);
-        uint32_t pk[16], dk[16];
+        tmem_load_2x32cols(t_s + chunk * 32, t_p + chunk * 32, sv, pv);
+        if (partial) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int c = chunk * 32 + e;
+            if (c > hi_c || c < lo_c) sv[e] = 0xff800000u;  // -inf
+          }
+        }
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           float pr[2], ds[2];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int c = chunk * 32 + e + h;  // query column within the tile
-            float x = bexp2(__uint_as_float(sv[e + h]) * c2 - s_lse[c]);
-            if (partial && !key_visible(p, m * kTile + c, key)) x = 0.f;
+            const float x = bexp2(__uint_as_float(sv[e + h]) * c2 - s_lse[c]);
             pr[h] = x;
             ds[h] = x * (__uint_as_float(pv[e + h]) - s_dlt[c]);
           }
-          pk[e >> 1] = bf16x2_rn(pr[0], pr[1]);
-          dk[e >> 1] = bf16x2_rn(ds[0], ds[1]);
+          pk[chunk][e >> 1] = bf16x2_rn(pr[0], pr[1]);
+          dk[chunk][e >> 1] = bf16x2_rn(ds[0], ds[1]);
         }
-        tmem_store_16cols(t_s + chunk * 16, pk);  // P^T over the first half of the S^T columns
-        tmem_store_16cols(t_p + chunk * 16, dk);  // dS^T over the first half of the dP^T columns
+      }
+#pragma unroll
+      for (int chunk = 0; chunk < 4; ++chunk) {
+        tmem_store_16cols(t_s + chunk * 16, pk[chunk]);  // P^T over the first half of the S^T columns
+        tmem_store_16cols(t_p + chunk * 16, dk[chunk]);  // dS^T over the first half of the dP^T columns
       }
       tmem_store_wait();
       tc_fence_before_sync();

@@ -439,6 +439,12 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
     bool pend = false;
     bool first_pv = true;
 
+    // The V tile with load index vn has landed (a tile this warp does not
+    // read must still be seen before this warp releases it).
+    auto wait_v_landed = [&](uint32_t vn) -> bool {
+      const uint32_t vslot = vn % L::kStages;
+      return wait_all(bar(L::kKVFull + vslot), (vn / L::kStages) & 1, code | (L::kKVFull + vslot));
+    };
     // O_t += P_t V for the V tile with load index vn.
     auto issue_pv = [&](uint32_t vn) -> bool {
       if (first_pv && items > 0 && !wait_all(bar(L::kOFree + t), (items - 1) & 1, code | (L::kOFree + t)))
@@ -467,7 +473,12 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
         ok = false;
         break;
       }
-      if (pend && !issue_pv(kv_n - 1)) {
+      if (pend) {
+        if (!issue_pv(kv_n - 1)) {
+          ok = false;
+          break;
+        }
+      } else if (j > it.lo_u && !wait_v_landed(kv_n - 1)) {
         ok = false;
         break;
       }
@@ -484,13 +495,19 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
         tc_commit_elect(bar(L::kSFull + t));
         pend = true;
       }
-      tc_commit_elect(bar(L::kKVEmpty + kslot));                                   // K_j read
+      // Each slot's empty barrier takes one arrival per MMA warp and phase.
+      // A warp releases a tile only after it has seen that tile land (for a
+      // tile this warp's MMAs do not read, wait_v_landed above), so its
+      // arrival for a load can only come after the load was issued, i.e.
+      // after the slot's previous phase completed: no warp ever arrives twice
+      // in one phase, even when its own tile is idle and it runs ahead.
       if (j > it.lo_u) tc_commit_elect(bar(L::kKVEmpty + (kv_n - 1) % L::kStages));  // V_{j-1} read
+      tc_commit_elect(bar(L::kKVEmpty + kslot));                                   // K_j read
       if (j == it.hi_u) tc_commit_elect(bar(L::kQEmpty));                          // Q read
       kv_n += 2;
     }
     if (!ok) break;
-    if (pend && !issue_pv(kv_n - 1)) break;
+    if (pend ? !issue_pv(kv_n - 1) : !wait_v_landed(kv_n - 1)) break;
     tc_commit_elect(bar(L::kKVEmpty + (kv_n - 1) % L::kStages));  // V_hi read
     if (first_pv && items > 0 && !wait_all(bar(L::kOFree + t), (items - 1) & 1, code | (L::kOFree + t))) break;
     tc_commit_elect(bar(L::kODone + t));
