@@ -38,6 +38,7 @@ namespace attn_sm100_bwd {
 using namespace attn_sm100;
 
 constexpr int kTile = 128;  // rows of every Q / dO / K / V tile
+constexpr int kHalf = 64;   // keys (dQ kernel) or queries (dK/dV kernel) per score half
 constexpr int kBwdThreads = 192;
 constexpr int kBwdLoaderWarp = 4;
 constexpr int kBwdMmaWarp = 5;
@@ -213,17 +214,20 @@ struct BwdSmem {
   static constexpr int kFixEmpty = 1;
   static constexpr int kRingFull = 2;
   static constexpr int kRingEmpty = kRingFull + kStages;
-  static constexpr int kSFull = kRingEmpty + kStages;
-  static constexpr int kPFull = kSFull + 1;
-  static constexpr int kAccDone = kPFull + 1;
+  static constexpr int kSFull = kRingEmpty + kStages;  // two: one per score half
+  static constexpr int kPFull = kSFull + 2;             // two: one per score half
+  static constexpr int kAccDone = kPFull + 2;
   static constexpr int kAccFree = kAccDone + 1;
   static constexpr int kFin = kAccFree + 1;
   static constexpr int kNumBars = kFin + 1;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
-  // TMEM columns: scores (or S^T), dP (or dP^T), then the accumulators.
-  static constexpr uint32_t kColS = 0, kColP = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
+  // TMEM columns: two buffers of 64-wide score halves, each S (or S^T) then
+  // dP (or dP^T), then the accumulators.
+  static constexpr uint32_t kColAcc0 = 256, kColAcc1 = 256 + D;
+  static __device__ __forceinline__ uint32_t col_s(int h) { return h * 128; }
+  static __device__ __forceinline__ uint32_t col_p(int h) { return h * 128 + 64; }
 };
 
 // Operand descriptors of a tile stored as 128 rows x D (K-major: the D axis
@@ -335,20 +339,36 @@ template <int D>
 __device__ __forceinline__ void dq_mma(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w) {
   using L = BwdSmem<D>;
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
-  constexpr uint32_t idesc_ss = idesc_bf16_f32(kTile, kTile, false);
+  constexpr uint32_t idesc_ss = idesc_bf16_f32(kTile, kHalf, false);  // 128 x 64 score halves
   constexpr uint32_t idesc_ts = idesc_bf16_f32(kTile, D, true);
-  const uint32_t t_s = tmem + L::kColS, t_p = tmem + L::kColP, t_acc = tmem + L::kColAcc0;
+  const uint32_t t_acc = tmem + L::kColAcc0;
   const uint64_t q_desc = kmajor_desc<D>(sbase + L::kFixOff);
   const uint64_t do_desc = kmajor_desc<D>(sbase + L::kFixOff + L::kTileBytes);
   const int code = (kBKernelDq << 12) | (kBRoleMma << 8);
-  uint32_t n = 0, ds_cnt = 0;
+  uint32_t n = 0;
+  uint32_t p_cnt0 = 0, p_cnt1 = 0;  // P / dS halves consumed, per half
   int items = 0;
   bool ok = true;
+  // dQ += dS_h K_h for half h of the key tile in ring slot `slot`.
+  auto issue_dq = [&](int h, uint32_t slot, bool first) -> bool {
+    if (!w.wait_warp(bar(L::kPFull + h), (h ? p_cnt1 : p_cnt0) & 1, code | (L::kPFull + h))) return false;
+    if (h) ++p_cnt1; else ++p_cnt0;
+    if (first && items > 0 && !w.wait_warp(bar(L::kAccFree), (items - 1) & 1, code | L::kAccFree)) return false;
+    tc_fence_after_sync();
+    const uint64_t kb = mnmajor_desc<D>(sbase + L::kRingOff + slot * 2 * L::kTileBytes) + ((h * kHalf * 128) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < kHalf / 16; ++kk)
+      mma_bf16_ts_elect(t_acc, tmem + L::col_s(h) + kk * 8, kb + ((kk * 2048) >> 4), idesc_ts,
+                        (kk > 0 || !first) ? 1u : 0u);
+    return true;
+  };
   for (int i = blockIdx.x; ok && i < p.num_items; i += gridDim.x, ++items) {
     const DqItem it = dq_item(p, i);
     if (!w.wait_warp(bar(L::kFixFull), items & 1, code | L::kFixFull)) break;
     tc_fence_after_sync();
-    for (int j = it.lo; j <= it.hi; ++j, ++n) {
+    uint32_t prev_slot = 0;
+    bool first_dq = true;
+    for (int j = it.lo; j <= it.hi && ok; ++j, ++n) {
       const uint32_t slot = n % L::kStages;
       const uint32_t kaddr = sbase + L::kRingOff + slot * 2 * L::kTileBytes;
       if (!w.wait_warp(bar(L::kRingFull + slot), (n / L::kStages) & 1, code | (L::kRingFull + slot))) {
@@ -356,32 +376,34 @@ __device__ __forceinline__ void dq_mma(const BwdParams& p, uint32_t sbase, uint3
         break;
       }
       tc_fence_after_sync();
-      const uint64_t k_desc = kmajor_desc<D>(kaddr), v_desc = kmajor_desc<D>(kaddr + L::kTileBytes);
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        // S_h = Q K_h^T and dP_h = dO V_h^T (keys 64h .. 64h+63 of the tile).
+        const uint64_t k_desc = kmajor_desc<D>(kaddr + h * kHalf * 128);
+        const uint64_t v_desc = kmajor_desc<D>(kaddr + L::kTileBytes + h * kHalf * 128);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = kmajor_off<D>(kk);
-        mma_bf16_ss_elect(t_s, q_desc + off, k_desc + off, idesc_ss, kk > 0 ? 1u : 0u);   // S = Q K^T
-        mma_bf16_ss_elect(t_p, do_desc + off, v_desc + off, idesc_ss, kk > 0 ? 1u : 0u);  // dP = dO V^T
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = kmajor_off<D>(kk);
+          mma_bf16_ss_elect(tmem + L::col_s(h), q_desc + off, k_desc + off, idesc_ss, kk > 0 ? 1u : 0u);
+          mma_bf16_ss_elect(tmem + L::col_p(h), do_desc + off, v_desc + off, idesc_ss, kk > 0 ? 1u : 0u);
+        }
+        tc_commit_elect(bar(L::kSFull + h));
+        if (j == it.hi && h == 1) tc_commit_elect(bar(L::kFixEmpty));  // Q, dO read
+        // dQ for the half before this one: (j, 0) now, or (j - 1, 1) at h = 0.
+        if (h == 1 || j > it.lo) {
+          if (!issue_dq(1 - h, h == 1 ? slot : prev_slot, first_dq)) {
+            ok = false;
+            break;
+          }
+          first_dq = false;
+          if (h == 0) tc_commit_elect(bar(L::kRingEmpty + prev_slot));  // previous K, V tile done
+        }
       }
-      tc_commit_elect(bar(L::kSFull));
-      if (j == it.hi) tc_commit_elect(bar(L::kFixEmpty));  // Q, dO read
-      if (!w.wait_warp(bar(L::kPFull), ds_cnt & 1, code | L::kPFull)) {
-        ok = false;
-        break;
-      }
-      ++ds_cnt;
-      if (j == it.lo && items > 0 && !w.wait_warp(bar(L::kAccFree), (items - 1) & 1, code | L::kAccFree)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after_sync();
-      const uint64_t kb_desc = mnmajor_desc<D>(kaddr);
-#pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk)  // dQ += dS K (dS in TMEM over the S columns)
-        mma_bf16_ts_elect(t_acc, t_s + kk * 8, kb_desc + ((kk * 2048) >> 4), idesc_ts, (kk > 0 || j > it.lo) ? 1u : 0u);
-      tc_commit_elect(bar(L::kRingEmpty + slot));
+      prev_slot = slot;
     }
     if (!ok) break;
+    if (!issue_dq(1, prev_slot, first_dq)) break;  // the item's last half
+    tc_commit_elect(bar(L::kRingEmpty + prev_slot));
     tc_commit_elect(bar(L::kAccDone));
   }
 }
@@ -393,11 +415,10 @@ __device__ __forceinline__ void dq_elem(const BwdParams& p, uint32_t sbase, uint
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
   const int r = warp * 32 + lane;  // row of the query tile = TMEM lane
   const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t t_s = tmem + lane_bits + L::kColS, t_p = tmem + lane_bits + L::kColP;
   const uint32_t t_acc = tmem + lane_bits + L::kColAcc0;
   const float c2 = p.scale_log2;
   const int code = (kBKernelDq << 12) | (kBRoleElem << 8);
-  uint32_t s_cnt = 0;
+  uint32_t s_cnt = 0;  // key tiles processed (each has both halves)
   int items = 0;
   for (int i = blockIdx.x; i < p.num_items; i += gridDim.x, ++items) {
     const DqItem it = dq_item(p, i);
@@ -407,50 +428,52 @@ __device__ __forceinline__ void dq_elem(const BwdParams& p, uint32_t sbase, uint
     const float lse2 = row_ok ? p.lse[bhrow] * kLog2e : 0.f;
     const float dlt = row_ok ? p.delta[bhrow] : 0.f;
     bool ok = true;
-    for (int j = it.lo; j <= it.hi; ++j) {
-      if (!w.wait_warp(bar(L::kSFull), s_cnt & 1, code | L::kSFull)) {
-        ok = false;
-        break;
-      }
-      ++s_cnt;
-      tc_fence_after_sync();
+    for (int j = it.lo; j <= it.hi && ok; ++j, ++s_cnt) {
       const bool partial = block_is_partial(p, it.m, j);
-      // Visible key columns of this row in the tile: lo_c <= c <= hi_c (only
-      // applied on partial tiles, where the masked scores become -inf).
-      const int j0 = j * kTile;
-      const int hi_c = row_ok ? min(p.N - 1, p.mask_kind == kBMaskFull ? p.N - 1 : row) - j0 : -1;
-      const int lo_c = (p.mask_kind == kBMaskWindow) ? row - p.window + 1 - j0 : 0;
-      // All loads before any store: dS (bf16, 64 columns) is kept in registers
-      // and written over the first half of the S columns at the end.
-      uint32_t packed[4][16];
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        if (!w.wait_warp(bar(L::kSFull + h), s_cnt & 1, code | (L::kSFull + h))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        // Visible key columns of this row in the half: lo_c <= c <= hi_c
+        // (applied on partial tiles, where masked scores become -inf).
+        const int j0 = j * kTile + h * kHalf;
+        const int hi_c = row_ok ? min(p.N - 1, p.mask_kind == kBMaskFull ? p.N - 1 : row) - j0 : -1;
+        const int lo_c = (p.mask_kind == kBMaskWindow) ? row - p.window + 1 - j0 : 0;
+        const uint32_t t_s = tmem + lane_bits + L::col_s(h), t_p = tmem + lane_bits + L::col_p(h);
+        uint32_t packed[2][16];
 #pragma unroll
-      for (int chunk = 0; chunk < 4; ++chunk) {
-        uint32_t sv[32], pv[32];
-        tmem_load_2x32cols(t_s + chunk * 32, t_p + chunk * 32, sv, pv);
-        if (partial) {
+        for (int chunk = 0; chunk < 2; ++chunk) {
+          uint32_t sv[32], pv[32];
+          tmem_load_2x32cols(t_s + chunk * 32, t_p + chunk * 32, sv, pv);
+          if (partial) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c = chunk * 32 + e;
-            if (c > hi_c || c < lo_c) sv[e] = 0xff800000u;  // -inf
+            for (int e = 0; e < 32; ++e) {
+              const int c = chunk * 32 + e;
+              if (c > hi_c || c < lo_c) sv[e] = 0xff800000u;  // -inf
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float ds[2];
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              const float pr = bexp2(__uint_as_float(sv[e + x]) * c2 - lse2);
+              ds[x] = pr * (__uint_as_float(pv[e + x]) - dlt);
+            }
+            packed[chunk][e >> 1] = bf16x2_rn(ds[0], ds[1]);
           }
         }
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float ds[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const float pr = bexp2(__uint_as_float(sv[e + h]) * c2 - lse2);
-            ds[h] = pr * (__uint_as_float(pv[e + h]) - dlt);
-          }
-          packed[chunk][e >> 1] = bf16x2_rn(ds[0], ds[1]);
-        }
+        // dS (bf16, 32 columns) over the first half of this half's S columns.
+        tmem_store_16cols(t_s, packed[0]);
+        tmem_store_16cols(t_s + 16, packed[1]);
+        tmem_store_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::kPFull + h));
       }
-#pragma unroll
-      for (int chunk = 0; chunk < 4; ++chunk) tmem_store_16cols(t_s + chunk * 16, packed[chunk]);
-      tmem_store_wait();
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::kPFull));
     }
     if (!ok) break;
     if (!w.wait_warp(bar(L::kAccDone), items & 1, code | L::kAccDone)) break;
@@ -544,21 +567,39 @@ template <int D>
 __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w) {
   using L = BwdSmem<D>;
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
-  constexpr uint32_t idesc_ss = idesc_bf16_f32(kTile, kTile, false);
+  constexpr uint32_t idesc_ss = idesc_bf16_f32(kTile, kHalf, false);  // 128 keys x 64 queries
   constexpr uint32_t idesc_ts = idesc_bf16_f32(kTile, D, true);
-  const uint32_t t_s = tmem + L::kColS, t_p = tmem + L::kColP;
   const uint32_t t_dv = tmem + L::kColAcc0, t_dk = tmem + L::kColAcc1;
   const uint64_t k_desc = kmajor_desc<D>(sbase + L::kFixOff);
   const uint64_t v_desc = kmajor_desc<D>(sbase + L::kFixOff + L::kTileBytes);
   const int code = (kBKernelDkdv << 12) | (kBRoleMma << 8);
-  uint32_t n = 0, p_cnt = 0;
+  uint32_t n = 0;
+  uint32_t p_cnt0 = 0, p_cnt1 = 0;  // P / dS halves consumed, per half
   int items = 0;
   bool ok = true;
+  // dV += P^T_h dO_h and dK += dS^T_h Q_h for query half h of ring slot `slot`.
+  auto issue_dkv = [&](int h, uint32_t slot, bool first) -> bool {
+    if (!w.wait_warp(bar(L::kPFull + h), (h ? p_cnt1 : p_cnt0) & 1, code | (L::kPFull + h))) return false;
+    if (h) ++p_cnt1; else ++p_cnt0;
+    if (first && items > 0 && !w.wait_warp(bar(L::kAccFree), (items - 1) & 1, code | L::kAccFree)) return false;
+    tc_fence_after_sync();
+    const uint32_t qaddr = sbase + L::kRingOff + slot * 2 * L::kTileBytes + h * kHalf * 128;
+    const uint64_t qb = mnmajor_desc<D>(qaddr), dob = mnmajor_desc<D>(qaddr + L::kTileBytes);
+#pragma unroll
+    for (int kk = 0; kk < kHalf / 16; ++kk) {
+      const uint32_t acc = (kk > 0 || !first) ? 1u : 0u;
+      mma_bf16_ts_elect(t_dv, tmem + L::col_s(h) + kk * 8, dob + ((kk * 2048) >> 4), idesc_ts, acc);
+      mma_bf16_ts_elect(t_dk, tmem + L::col_p(h) + kk * 8, qb + ((kk * 2048) >> 4), idesc_ts, acc);
+    }
+    return true;
+  };
   for (int i = blockIdx.x; ok && i < p.num_items; i += gridDim.x, ++items) {
     const DkvItem it = dkv_item(p, i);
     if (!w.wait_warp(bar(L::kFixFull), items & 1, code | L::kFixFull)) break;
     tc_fence_after_sync();
-    for (int s = 0; s < it.steps; ++s, ++n) {
+    uint32_t prev_slot = 0;
+    bool first = true;
+    for (int s = 0; s < it.steps && ok; ++s, ++n) {
       const uint32_t slot = n % L::kStages;
       const uint32_t qaddr = sbase + L::kRingOff + slot * 2 * L::kTileBytes;
       if (!w.wait_warp(bar(L::kRingFull + slot), (n / L::kStages) & 1, code | (L::kRingFull + slot))) {
@@ -566,35 +607,33 @@ __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint
         break;
       }
       tc_fence_after_sync();
-      const uint64_t q_desc = kmajor_desc<D>(qaddr), do_desc = kmajor_desc<D>(qaddr + L::kTileBytes);
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        // S^T_h = K Q_h^T and dP^T_h = V dO_h^T (queries 64h .. 64h+63 of the tile).
+        const uint64_t q_desc = kmajor_desc<D>(qaddr + h * kHalf * 128);
+        const uint64_t do_desc = kmajor_desc<D>(qaddr + L::kTileBytes + h * kHalf * 128);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = kmajor_off<D>(kk);
-        mma_bf16_ss_elect(t_s, k_desc + off, q_desc + off, idesc_ss, kk > 0 ? 1u : 0u);   // S^T = K Q^T
-        mma_bf16_ss_elect(t_p, v_desc + off, do_desc + off, idesc_ss, kk > 0 ? 1u : 0u);  // dP^T = V dO^T
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = kmajor_off<D>(kk);
+          mma_bf16_ss_elect(tmem + L::col_s(h), k_desc + off, q_desc + off, idesc_ss, kk > 0 ? 1u : 0u);
+          mma_bf16_ss_elect(tmem + L::col_p(h), v_desc + off, do_desc + off, idesc_ss, kk > 0 ? 1u : 0u);
+        }
+        tc_commit_elect(bar(L::kSFull + h));
+        if (s == it.steps - 1 && h == 1) tc_commit_elect(bar(L::kFixEmpty));  // K, V read
+        if (h == 1 || s > 0) {
+          if (!issue_dkv(1 - h, h == 1 ? slot : prev_slot, first)) {
+            ok = false;
+            break;
+          }
+          first = false;
+          if (h == 0) tc_commit_elect(bar(L::kRingEmpty + prev_slot));  // previous Q, dO tile done
+        }
       }
-      tc_commit_elect(bar(L::kSFull));
-      if (s == it.steps - 1) tc_commit_elect(bar(L::kFixEmpty));  // K, V read
-      if (!w.wait_warp(bar(L::kPFull), p_cnt & 1, code | L::kPFull)) {
-        ok = false;
-        break;
-      }
-      ++p_cnt;
-      if (s == 0 && items > 0 && !w.wait_warp(bar(L::kAccFree), (items - 1) & 1, code | L::kAccFree)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after_sync();
-      const uint64_t dob_desc = mnmajor_desc<D>(qaddr + L::kTileBytes), qb_desc = mnmajor_desc<D>(qaddr);
-#pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk) {
-        const uint32_t acc = (kk > 0 || s > 0) ? 1u : 0u;
-        mma_bf16_ts_elect(t_dv, t_s + kk * 8, dob_desc + ((kk * 2048) >> 4), idesc_ts, acc);  // dV += P^T dO
-        mma_bf16_ts_elect(t_dk, t_p + kk * 8, qb_desc + ((kk * 2048) >> 4), idesc_ts, acc);   // dK += dS^T Q
-      }
-      tc_commit_elect(bar(L::kRingEmpty + slot));
+      prev_slot = slot;
     }
     if (!ok) break;
+    if (!issue_dkv(1, prev_slot, first)) break;  // the item's last half
+    tc_commit_elect(bar(L::kRingEmpty + prev_slot));
     tc_commit_elect(bar(L::kAccDone));
   }
 }
@@ -606,7 +645,6 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
   const int r = warp * 32 + lane;  // key row of the tile = TMEM lane
   const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t t_s = tmem + lane_bits + L::kColS, t_p = tmem + lane_bits + L::kColP;
   const uint32_t t_dv = tmem + lane_bits + L::kColAcc0, t_dk = tmem + lane_bits + L::kColAcc1;
   // This warp's copy of the step's log2-scaled LSE and D of the 128 query rows.
   float* s_lse = reinterpret_cast<float*>(__cvta_shared_to_generic(sbase + L::kVecOff)) + warp * 2 * kTile;
@@ -619,7 +657,7 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
     const DkvItem it = dkv_item(p, i);
     const int key = it.n * kTile + r;
     bool ok = true;
-    for (int s = 0; s < it.steps; ++s) {
+    for (int s = 0; s < it.steps && ok; ++s, ++s_cnt) {
       int hq, m;
       dkv_step(p, it, s, hq, m);
       {
@@ -633,57 +671,57 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
         }
         __syncwarp();
       }
-      if (!w.wait_warp(bar(L::kSFull), s_cnt & 1, code | L::kSFull)) {
-        ok = false;
-        break;
-      }
-      ++s_cnt;
-      tc_fence_after_sync();
       const bool partial = block_is_partial(p, m, it.n);
-      // Query columns that see this key: lo_c <= c <= hi_c (only applied on
-      // partial tiles, where the masked scores become -inf).
-      const int q0 = m * kTile;
-      const int hi_c = (key < p.N)
-                           ? min(p.N - 1, p.mask_kind == kBMaskWindow ? key + p.window - 1 : p.N - 1) - q0
-                           : -1;
-      const int lo_c = (p.mask_kind == kBMaskFull) ? 0 : key - q0;
-      // All loads before any store: P^T and dS^T (bf16, 64 columns each) are
-      // kept in registers and written over the first halves at the end.
-      uint32_t pk[4][16], dk[4][16];
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        if (!w.wait_warp(bar(L::kSFull + h), s_cnt & 1, code | (L::kSFull + h))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        // Query columns of this half that see the key: lo_c <= c <= hi_c
+        // (applied on partial tiles, where masked scores become -inf).
+        const int q0 = m * kTile + h * kHalf;
+        const int hi_c =
+            (key < p.N) ? min(p.N - 1, p.mask_kind == kBMaskWindow ? key + p.window - 1 : p.N - 1) - q0 : -1;
+        const int lo_c = (p.mask_kind == kBMaskFull) ? 0 : key - q0;
+        const uint32_t t_s = tmem + lane_bits + L::col_s(h), t_p = tmem + lane_bits + L::col_p(h);
+        uint32_t pk[2][16], dk[2][16];
 #pragma unroll
-      for (int chunk = 0; chunk < 4; ++chunk) {
-        uint32_t sv[32], pv[32];
-        tmem_load_2x32cols(t_s + chunk * 32, t_p + chunk * 32, sv, pv);
-        if (partial) {
+        for (int chunk = 0; chunk < 2; ++chunk) {
+          uint32_t sv[32], pv[32];
+          tmem_load_2x32cols(t_s + chunk * 32, t_p + chunk * 32, sv, pv);
+          if (partial) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c = chunk * 32 + e;
-            if (c > hi_c || c < lo_c) sv[e] = 0xff800000u;  // -inf
+            for (int e = 0; e < 32; ++e) {
+              const int c = chunk * 32 + e;
+              if (c > hi_c || c < lo_c) sv[e] = 0xff800000u;  // -inf
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float pr[2], ds[2];
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              const int c = h * kHalf + chunk * 32 + e + x;  // query column within the tile
+              pr[x] = bexp2(__uint_as_float(sv[e + x]) * c2 - s_lse[c]);
+              ds[x] = pr[x] * (__uint_as_float(pv[e + x]) - s_dlt[c]);
+            }
+            pk[chunk][e >> 1] = bf16x2_rn(pr[0], pr[1]);
+            dk[chunk][e >> 1] = bf16x2_rn(ds[0], ds[1]);
           }
         }
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pr[2], ds[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int c = chunk * 32 + e + h;  // query column within the tile
-            const float x = bexp2(__uint_as_float(sv[e + h]) * c2 - s_lse[c]);
-            pr[h] = x;
-            ds[h] = x * (__uint_as_float(pv[e + h]) - s_dlt[c]);
-          }
-          pk[chunk][e >> 1] = bf16x2_rn(pr[0], pr[1]);
-          dk[chunk][e >> 1] = bf16x2_rn(ds[0], ds[1]);
-        }
+        // P^T and dS^T (bf16, 32 columns each) over the first halves of this
+        // half's S^T and dP^T columns.
+        tmem_store_16cols(t_s, pk[0]);
+        tmem_store_16cols(t_s + 16, pk[1]);
+        tmem_store_16cols(t_p, dk[0]);
+        tmem_store_16cols(t_p + 16, dk[1]);
+        tmem_store_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::kPFull + h));
       }
-#pragma unroll
-      for (int chunk = 0; chunk < 4; ++chunk) {
-        tmem_store_16cols(t_s + chunk * 16, pk[chunk]);  // P^T over the first half of the S^T columns
-        tmem_store_16cols(t_p + chunk * 16, dk[chunk]);  // dS^T over the first half of the dP^T columns
-      }
-      tmem_store_wait();
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::kPFull));
     }
     if (!ok) break;
     if (!w.wait_warp(bar(L::kAccDone), items & 1, code | L::kAccDone)) break;
@@ -718,8 +756,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
       mbar_init(bar(L::kRingFull + s), 1);
       mbar_init(bar(L::kRingEmpty + s), 1);
     }
-    mbar_init(bar(L::kSFull), 1);
-    mbar_init(bar(L::kPFull), 4);    // one arrival per elementwise warp
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(bar(L::kSFull + h), 1);
+      mbar_init(bar(L::kPFull + h), 4);  // one arrival per elementwise warp
+    }
     mbar_init(bar(L::kAccDone), 1);
     mbar_init(bar(L::kAccFree), 4);  // one arrival per elementwise warp
     mbar_init(bar(L::kFin), 1);
