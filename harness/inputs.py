@@ -112,3 +112,119 @@ def make_dout(B, Hq, N, d, seed, device="cpu", dtype=torch.bfloat16):
     gen = torch.Generator(device=device)
     gen.manual_seed(int(seed) + 7919)
     return torch.randn((B, Hq, N, d), generator=gen, device=device, dtype=torch.float32).to(dtype)
+
+
+# ---------------------------------------------------------------- decoding
+# Decoding workloads: the new token(s) of each sequence attend to a paged KV
+# cache.  Shapes follow the pages' long-context figures (128k context, d=128,
+# 32 heads; GQA with 64 query heads over 8 KV heads; a 4096-token window);
+# page_size 16 tokens.  Ragged batches draw each sequence length uniformly in
+# [L_min, L_max].
+@dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    d: int
+    L_min: int
+    L_max: int
+    page_size: int
+    mask: str
+    window: Optional[int]
+    seed: int
+    rolling: bool = False   # pages wholly before the window are not allocated (table entry -1)
+
+    @property
+    def mask_kind(self) -> int:
+        return MASK_NAMES[self.mask]
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.d))
+
+    def as_dict(self) -> dict:
+        return asdict(self)
+
+
+DECODE_WORKLOADS = {
+    "decode_gqa": DecodeWorkload("decode_gqa", 1, 64, 8, 1, 128, 131072, 131072, 16, "causal", None, 10),
+    "decode_mha": DecodeWorkload("decode_mha", 16, 32, 32, 1, 128, 8192, 32768, 16, "causal", None, 11),
+    "decode_swa": DecodeWorkload("decode_swa", 32, 32, 8, 1, 128, 65536, 131072, 16, "sliding_window", 4096,
+                                 12, rolling=True),
+    "decode_spec": DecodeWorkload("decode_spec", 8, 64, 8, 4, 128, 16384, 32768, 64, "causal", None, 13),
+}
+
+
+def make_seq_lens(B: int, L_min: int, L_max: int, seed: int) -> np.ndarray:
+    """Sequence lengths: B integers uniform in [L_min, L_max] (numpy generator
+    seeded with ``seed``)."""
+    rng = np.random.default_rng(int(seed))
+    return rng.integers(L_min, L_max + 1, size=B, dtype=np.int64)
+
+
+def make_paged_kv(B, Hq, Hkv, Nq, d, seq_lens, page_size, seed, device="cpu", keep_from=None,
+                  fill=None, extra_pages=0, table_width=None, dtype=torch.bfloat16):
+    """Draw a decoding step's inputs with its KV cache in pages.
+
+    Sequence b keeps logical pages ``keep_from[b] // page_size`` ..
+    ``(seq_lens[b] - 1) // page_size`` (``keep_from`` defaults to 0); every
+    other table entry is -1.  Physical pages are handed out in the order of a
+    seeded random permutation, so consecutive logical pages are scattered over
+    the pool, and ``extra_pages`` unused pages are added to it.
+
+    Draw order on a ``torch.Generator`` seeded with ``seed``: q [B,Hq,Nq,d],
+    k_cache and v_cache [num_pages,Hkv,page_size,d] as fp32 N(0,1) cast to
+    bf16, then the page permutation.  With ``fill`` given, every cache slot
+    that holds no kept position (slots past the end of a sequence's last page,
+    the extra pages) is set to ``fill`` (e.g. NaN to show it is never read).
+    Returns a dict of tensors: q, k_cache, v_cache, block_table (int32
+    [B, table_width]), seq_lens (int32 [B]).
+    """
+    seq_lens = np.asarray(seq_lens, dtype=np.int64)
+    keep_from = np.zeros(B, dtype=np.int64) if keep_from is None else np.asarray(keep_from, dtype=np.int64)
+    first = keep_from // page_size
+    last = (seq_lens - 1) // page_size
+    counts = last - first + 1
+    num_pages = int(counts.sum()) + int(extra_pages)
+    width = int(last.max()) + 1 if table_width is None else int(table_width)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    q = torch.randn((B, Hq, Nq, d), generator=gen, device=device, dtype=torch.float32).to(dtype)
+    k_cache = torch.randn((num_pages, Hkv, page_size, d), generator=gen, device=device,
+                          dtype=torch.float32).to(dtype)
+    v_cache = torch.randn((num_pages, Hkv, page_size, d), generator=gen, device=device,
+                          dtype=torch.float32).to(dtype)
+    perm = torch.randperm(num_pages, generator=gen, device=device).cpu().numpy()
+    table = np.full((B, width), -1, dtype=np.int32)
+    used = np.zeros(num_pages, dtype=np.int64)  # kept slots per physical page (fill bookkeeping)
+    nxt = 0
+    for b in range(B):
+        for lp in range(int(first[b]), int(last[b]) + 1):
+            phys = int(perm[nxt])
+            nxt += 1
+            table[b, lp] = phys
+            used[phys] = min(page_size, int(seq_lens[b]) - lp * page_size)
+    if fill is not None:
+        for phys in range(num_pages):
+            if used[phys] < page_size:
+                k_cache[phys, :, used[phys]:, :] = fill
+                v_cache[phys, :, used[phys]:, :] = fill
+    return {
+        "q": q, "k_cache": k_cache, "v_cache": v_cache,
+        "block_table": torch.from_numpy(table).to(device),
+        "seq_lens": torch.from_numpy(seq_lens.astype(np.int32)).to(device),
+    }
+
+
+def make_decode_workload(w: DecodeWorkload, device="cpu", fill=None):
+    """Inputs of a decoding workload (lengths from ``make_seq_lens`` with the
+    workload's seed; for a rolling window the pages before position
+    L_b - Nq - w + 1 are not allocated)."""
+    lens = make_seq_lens(w.B, w.L_min, w.L_max, w.seed)
+    keep = None
+    if w.rolling:
+        keep = np.maximum(lens - w.Nq - w.window + 1, 0)
+    return make_paged_kv(w.B, w.Hq, w.Hkv, w.Nq, w.d, lens, w.page_size, w.seed, device=device,
+                         keep_from=keep, fill=fill)
