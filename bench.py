@@ -7,10 +7,13 @@ visible (query, key) pair.  Inputs (384 MiB of q, k, v) are larger than the
 126 MB L2, so no flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload dense|gqa|swa|long|tiny] [--no-cpu-baseline] [--pass fwd|bwd]
+                  [--workload dense|gqa|swa|long|tiny] [--no-cpu-baseline] [--pass fwd|bwd|decode]
 
 ``--pass bwd`` times the backward pass instead (one GPU; 10*d FLOPs per visible
-pair, the five products of the gradient).
+pair, the five products of the gradient).  ``--pass decode`` times one decoding
+step against a paged KV cache (``--workload decode_gqa|decode_mha|decode_swa|
+decode_spec``; one GPU; GB/s of algorithmic bytes against the measured HBM
+bandwidth).
 
 With --gpus N > 1 the script runs under torchrun, one rank per GPU; every rank
 runs its own shard of the global batch (weak scaling, no data-path collective)
@@ -36,7 +39,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from harness.inputs import WORKLOADS, make_qkv, sample_rows  # noqa: E402
+from harness.inputs import DECODE_WORKLOADS, WORKLOADS, make_qkv, sample_rows  # noqa: E402
 
 METRIC = "attention fwd TFLOP/s (bf16, causal/window-adjusted) and % of B200 dense peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -421,25 +424,172 @@ def run_backward(args, w):
     print(json.dumps(line), flush=True)
 
 
+DEC_METRIC = "attention decode GB/s (bf16 paged KV cache, algorithmic bytes) and % of measured HBM bandwidth"
+
+
+def decode_bytes(w, lens) -> int:
+    """Algorithmic bytes of one decoding step: K and V (bf16) of every position
+    a step's queries can see (from max(0, L - Nq - window + 1) under a window,
+    else from 0, to L - 1) for each KV head, plus q and out (bf16) and lse."""
+    keys = 0
+    for L in (int(x) for x in lens):
+        lo = max(0, L - w.Nq - w.window + 1) if w.mask == "sliding_window" else 0
+        keys += L - lo
+    return 2 * 2 * w.d * w.Hkv * keys + w.B * w.Hq * w.Nq * (2 * 2 * w.d + 4)
+
+
+def decode_cpu_sample(w, inp, seqs):
+    """The fp64 decoding oracle on the sequences ``seqs`` (host copies made
+    outside the timed region); returns (seconds, algorithmic bytes, threads)."""
+    from threadpoolctl import threadpool_info
+    from dataclasses import replace
+    from oracle import attention_decode_fp64 as DO
+    table = inp["block_table"].cpu().numpy()
+    lens = inp["seq_lens"].cpu().numpy()
+    used = sorted({int(pg) for b in seqs for pg in table[b] if pg >= 0})
+    remap = {pg: i for i, pg in enumerate(used)}
+    idx = torch.as_tensor(used, dtype=torch.long, device=inp["k_cache"].device)
+    kc = inp["k_cache"].index_select(0, idx).float().cpu().numpy()
+    vc = inp["v_cache"].index_select(0, idx).float().cpu().numpy()
+    sub = np.array([[remap.get(int(pg), -1) for pg in table[b]] for b in seqs], dtype=np.int64)
+    q = inp["q"][list(seqs)].float().cpu().numpy()
+    t0 = time.perf_counter()
+    DO.decode_attention(q, kc, vc, sub, lens[list(seqs)], w.scale, w.mask_kind, w.window)
+    dt = time.perf_counter() - t0
+    nbytes = decode_bytes(replace(w, B=len(seqs)), lens[list(seqs)])
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return dt, nbytes, threads
+
+
+def run_decode(args, w):
+    """Decoding step on one GPU: each step is one attn_decode call (the
+    decoding kernel, plus the split merge when the step uses splits) over the
+    workload's paged KV cache, resident in HBM."""
+    from harness.inputs import make_decode_workload
+    from exact_io_aware_72_b200 import decode, decode_num_splits, decode_workspace_bytes
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    inp = make_decode_workload(w, device=device)
+    lens = inp["seq_lens"].cpu().numpy()
+    max_len = int(lens.max())
+    splits = args.splits or decode_num_splits(w.B, w.Hq, w.Hkv, w.Nq, max_len, w.mask, w.window)
+    out = torch.empty_like(inp["q"])
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=device)
+    ws_bytes = decode_workspace_bytes(w.B, w.Hq, w.Nq, w.d, splits)
+    ws = torch.empty(max(ws_bytes // 4, 1), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    nbytes = decode_bytes(w, lens)
+
+    def step(q=inp["q"], bt=inp["block_table"], sl=inp["seq_lens"]):
+        decode(q, inp["k_cache"], inp["v_cache"], bt, sl, scale=w.scale, mask=w.mask, window=w.window,
+               num_splits=splits, out=out, lse=lse, workspace=ws, stream=stream)
+
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    clocks.mark(0)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    evs[0].record(stream)
+    for i in range(args.steps):
+        step()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize(device)
+    clocks.mark(1)
+    per_step_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    total_ms = evs[0].elapsed_time(evs[-1])
+    clk = clocks.stop()
+
+    # End to end: the step's new inputs (q, page table, lengths) from pinned host
+    # memory, the result (out, lse) back; the KV cache stays resident in HBM.
+    hq, hbt, hsl = (t.cpu().pin_memory() for t in (inp["q"], inp["block_table"], inp["seq_lens"]))
+    ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    dq, dbt, dsl = torch.empty_like(inp["q"]), torch.empty_like(inp["block_table"]), torch.empty_like(inp["seq_lens"])
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dbt.copy_(hbt, non_blocking=True)
+        dsl.copy_(hsl, non_blocking=True)
+        step(dq, dbt, dsl)
+        ho.copy_(out, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    e2e_steps = max(3, min(args.steps, 20))
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e0.elapsed_time(e1)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hbt, hsl))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["hbm_gbs"])
+    achieved = nbytes / (statistics.mean(per_step_ms) / 1e3) / 1e9
+    line = {
+        "metric": DEC_METRIC, "pass": "decode", "value": nbytes * args.steps / (total_ms / 1e3) / 1e9,
+        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "d": w.d,
+                   "seq_len_min": int(lens.min()), "seq_len_max": max_len, "page_size": w.page_size,
+                   "mask": w.mask, "window": w.window, "rolling_buffer": w.rolling, "num_splits": splits,
+                   "bytes_per_step": nbytes, "l2": "KV cache larger than L2 (no flush)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
+                     "note": "achieved over the whole step (decoding kernel plus split merge)"},
+        "gpu_launches": args.steps * (2 if splits > 1 else 1),
+        "launch_ms": {"median": statistics.median(per_step_ms), "best": min(per_step_ms)},
+        "clocks": clk,
+        "e2e": {"value": nbytes * e2e_steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+    }
+    if not args.no_cpu_baseline:
+        seqs = [0]
+        dt, nb, threads = decode_cpu_sample(w, inp, seqs)
+        line["cpu_baseline"] = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                "sample": f"sequence 0 of the {w.name} workload, all heads "
+                                          f"(fp64 NumPy, page-table gather and scores materialised), {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="dense")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS), default=None,
+                    help="default: dense (fwd, bwd) or decode_gqa (decode)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--shape", default=None,
                     help="B,Hq,Hkv,N,d: run this shape instead of a named workload (profiling sweeps)")
     ap.add_argument("--mask", choices=["full", "causal", "sliding_window"], default=None)
     ap.add_argument("--window", type=int, default=None)
-    ap.add_argument("--pass", dest="which", choices=["fwd", "bwd"], default="fwd",
-                    help="bwd: time the backward pass (one GPU) instead of the forward")
+    ap.add_argument("--pass", dest="which", choices=["fwd", "bwd", "decode"], default="fwd",
+                    help="bwd: the backward pass; decode: a paged-KV decoding step (one GPU each)")
+    ap.add_argument("--splits", type=int, default=0, help="decode: KV splits per sequence (0 = suggested)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    w = WORKLOADS[args.workload]
+    if args.which == "decode":
+        name = args.workload or "decode_gqa"
+        if name not in DECODE_WORKLOADS:
+            ap.error("--pass decode takes a decode_* workload")
+        run_decode(args, DECODE_WORKLOADS[name])
+        return
+    if args.workload in DECODE_WORKLOADS:
+        ap.error("decode_* workloads need --pass decode")
+    w = WORKLOADS[args.workload or "dense"]
     if args.shape or args.mask:
         from dataclasses import replace
         B, Hq, Hkv, N, d = (int(x) for x in args.shape.split(",")) if args.shape else (w.B, w.Hq, w.Hkv, w.N, w.d)

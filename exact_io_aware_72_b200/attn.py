@@ -19,7 +19,9 @@ STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3:
 ATTN_ERR_TIMEOUT = 5
 LIB_NAME = "libattn_b200.so"
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_status_string", "attn_debug_error", "attn_fwd_num_work_items",
-           "attn_bwd", "attn_bwd_ex", "attn_bwd_workspace_bytes", "attn_bwd_debug_error")
+           "attn_bwd", "attn_bwd_ex", "attn_bwd_workspace_bytes", "attn_bwd_debug_error",
+           "attn_decode", "attn_decode_ex", "attn_decode_workspace_bytes", "attn_decode_num_splits",
+           "attn_decode_debug_error")
 
 _lib = None
 
@@ -69,6 +71,17 @@ def load_library():
     lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_bwd_debug_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.attn_bwd_debug_error.restype = ctypes.c_int
+    dec_args = [vp] * 8 + [ctypes.c_size_t] + [i64] * 9 + [ctypes.c_float, ctypes.c_int, i64, vp]
+    lib.attn_decode.argtypes = dec_args
+    lib.attn_decode.restype = ctypes.c_int
+    lib.attn_decode_ex.argtypes = dec_args + [ctypes.POINTER(FwdOptions)]
+    lib.attn_decode_ex.restype = ctypes.c_int
+    lib.attn_decode_workspace_bytes.argtypes = [i64, i64, i64, i64, i64]
+    lib.attn_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_decode_num_splits.argtypes = [i64, i64, i64, i64, i64, ctypes.c_int, i64]
+    lib.attn_decode_num_splits.restype = i64
+    lib.attn_decode_debug_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    lib.attn_decode_debug_error.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -181,6 +194,95 @@ def bwd_debug_error(stream: Optional[torch.cuda.Stream] = None, device=None) -> 
     code = ctypes.c_int(0)
     with torch.cuda.device(stream.device):
         st = lib.attn_bwd_debug_error(ctypes.c_void_p(stream.cuda_stream), ctypes.byref(code))
+    return st, code.value
+
+
+def decode_num_splits(B, Hq, Hkv, Nq, max_seq_len, mask="causal", window=None) -> int:
+    """Suggested split count for a decoding step (host-only; see include/attn.h)."""
+    n = int(load_library().attn_decode_num_splits(B, Hq, Hkv, Nq, int(max_seq_len), MASKS[mask],
+                                                   int(window) if window is not None else 0))
+    if n < 1:
+        raise ValueError("invalid decoding sizes")
+    return n
+
+
+def decode_workspace_bytes(B, Hq, Nq, d, num_splits) -> int:
+    return int(load_library().attn_decode_workspace_bytes(B, Hq, Nq, d, int(num_splits)))
+
+
+def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_table: torch.Tensor,
+           seq_lens: torch.Tensor, max_seq_len: Optional[int] = None, scale: Optional[float] = None,
+           mask: str = "causal", window: Optional[int] = None, num_splits: Optional[int] = None,
+           out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+           workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+           wait_timeout_ns: int = 0, grid_ctas: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One decoding step against a paged KV cache: returns (out bf16 [B,Hq,Nq,d],
+    lse fp32 [B,Hq,Nq]).
+
+    q: [B,Hq,Nq,d] bf16 (the new tokens, the last Nq positions of each
+    sequence); k_cache/v_cache: [num_pages,Hkv,page_size,d] bf16;
+    block_table: [B,max_pages] int32; seq_lens: [B] int32 cached positions per
+    sequence (new tokens included).  ``max_seq_len`` (a host-side upper bound
+    of seq_lens, default max_pages*page_size) only picks the default
+    ``num_splits``.  The fp32 workspace for the splits' partial results is
+    allocated here when not given.
+    """
+    lib = load_library()
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(block_table, "block_table", torch.int32, 2)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hq, Nq, d = q.shape
+    num_pages, Hkv, page_size, dk = k_cache.shape
+    if dk != d or tuple(v_cache.shape) != tuple(k_cache.shape) or block_table.shape[0] != B \
+            or seq_lens.shape[0] != B:
+        raise ValueError("q, cache, block_table and seq_lens shapes disagree")
+    if mask not in MASKS:
+        raise ValueError(f"mask must be one of {sorted(MASKS)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    max_pages = block_table.shape[1]
+    if max_seq_len is None:
+        max_seq_len = max_pages * page_size
+    if num_splits is None:
+        num_splits = decode_num_splits(B, Hq, Hkv, Nq, max_seq_len, mask, window)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    ws_bytes = decode_workspace_bytes(B, Hq, Nq, d, num_splits)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes // 4, dtype=torch.float32, device=q.device)
+    ws_ptr, ws_len = 0, 0
+    if workspace is not None:
+        if not (workspace.is_cuda and workspace.is_contiguous()):
+            raise ValueError("workspace must be a contiguous CUDA tensor")
+        ws_ptr, ws_len = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    opts = FwdOptions(int(wait_timeout_ns), 0, int(grid_ctas))
+    with torch.cuda.device(q.device):
+        st = lib.attn_decode_ex(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
+                                seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(), ws_ptr, ws_len,
+                                B, Hq, Hkv, Nq, d, num_pages, page_size, max_pages, int(num_splits),
+                                float(scale), MASKS[mask], int(window) if window is not None else 0,
+                                ctypes.c_void_p(stream.cuda_stream), ctypes.byref(opts))
+    if st != 0:
+        raise AttnError(st, "attn_decode")
+    return out, lse
+
+
+def decode_debug_error(stream: Optional[torch.cuda.Stream] = None, device=None) -> Tuple[int, int]:
+    """Synchronise and read/clear the decoding kernel's error word: (status, raw code)."""
+    lib = load_library()
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    code = ctypes.c_int(0)
+    with torch.cuda.device(stream.device):
+        st = lib.attn_decode_debug_error(ctypes.c_void_p(stream.cuda_stream), ctypes.byref(code))
     return st, code.value
 
 

@@ -1,5 +1,5 @@
 /*
- * Exact attention forward and backward for NVIDIA B200 (sm_100a): C ABI.
+ * Exact attention forward, backward and paged-KV decoding for NVIDIA B200 (sm_100a): C ABI.
  *
  * Computes, for every batch b, query head h and query row i,
  *
@@ -156,6 +156,77 @@ size_t attn_bwd_workspace_bytes(int64_t B, int64_t Hq, int64_t N);
 
 /* attn_debug_error for the backward kernels' error word (same contract). */
 int attn_bwd_debug_error(cudaStream_t stream, int* device_code);
+/*
+ * attn_decode: enqueue one decoding step on `stream`: the Nq new tokens of each of B
+ * sequences attend to that sequence's cached keys and values, which are stored in
+ * fixed-size pages reached through a per-sequence page table ("Efficient attention:
+ * long context and sub-quadratic variants", stanleyjacob.dev, section "FlashAttention:
+ * exact attention, IO-aware", PagedAttention paragraph; "Efficient Attention",
+ * giftedprocrastinator.com, section "What it does": the KV cache keeps past keys and
+ * values so a new token does not recompute them). Nothing is approximated: the result is
+ * the masked softmax attention of attn_fwd for the new tokens' rows.
+ *
+ * With L_b = seq_lens[b] cached positions (the new tokens included), new token t of
+ * sequence b is at position L_b - Nq + t and sees cached positions j with
+ *   ATTN_MASK_FULL            0 <= j < L_b;
+ *   ATTN_MASK_CAUSAL          j <= L_b - Nq + t;
+ *   ATTN_MASK_SLIDING_WINDOW  L_b - Nq + t - window < j <= L_b - Nq + t.
+ * Position j of sequence b lives in physical page block_table[b][j / page_size], slot
+ * j % page_size. Only pages holding positions from lo_b = max(0, L_b - Nq - window + 1)
+ * (0 without a window) to L_b - 1 are looked up or read: under a sliding window a caller
+ * may recycle older pages and leave their table entries stale (a rolling window buffer);
+ * slots past L_b in the last page may hold anything.
+ *
+ *   q            device, bf16, [B, Hq, Nq, d], contiguous, 16-byte aligned
+ *   k_cache      device, bf16, [num_pages, Hkv, page_size, d], contiguous, 16-byte aligned
+ *   v_cache      device, bf16, same shape as k_cache
+ *   block_table  device, int32, [B, max_pages_per_seq], 4-byte aligned
+ *   seq_lens     device, int32, [B], 4-byte aligned; Nq <= seq_lens[b] <= max_pages_per_seq *
+ *                page_size (violations are reported by attn_decode_debug_error as
+ *                ATTN_ERR_INVALID_ARG and leave those rows zero with lse = -inf)
+ *   out          device, bf16, [B, Hq, Nq, d], 16-byte aligned; fully overwritten
+ *   lse          device, fp32, [B, Hq, Nq], 4-byte aligned; natural-log normaliser of each row
+ *   workspace    device, 16-byte aligned, at least attn_decode_workspace_bytes(B, Hq, Nq, d,
+ *                num_splits) bytes (none needed, may be NULL, when num_splits == 1); holds the
+ *                splits' partial results until the merge launch of the same call has read them
+ *   Hq % Hkv == 0; query head h reads KV head h / (Hq / Hkv); d in {64, 128};
+ *   page_size in {16, 32, 64, 128, 256}
+ *   num_splits   1..4096: each sequence's visible key range is cut into this many parts
+ *                processed in parallel and merged by their log-sum-exp
+ *                (attn_decode_num_splits suggests one)
+ *   scale, mask_kind, window, stream: as attn_fwd
+ *
+ * Ownership: the caller owns every buffer; the library allocates nothing and never
+ * synchronises. Outputs and the workspace must not overlap each other or the inputs
+ * (ATTN_ERR_INVALID_ARG). A page-table entry outside [0, num_pages) that the step needs
+ * is reported by attn_decode_debug_error as ATTN_ERR_INVALID_ARG (the step's result is
+ * then undefined, but nothing outside the given buffers is read). Errors, bounded waits
+ * and ATTN_ERR_TIMEOUT as attn_fwd.
+ */
+int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                const int32_t* seq_lens, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t d,
+                int64_t num_pages, int64_t page_size, int64_t max_pages_per_seq, int64_t num_splits,
+                float scale, int mask_kind, int64_t window, cudaStream_t stream);
+/* attn_decode with options (wait bound and CTA count as for attn_fwd_ex; inject_stall
+   is ignored); opts may be NULL. */
+int attn_decode_ex(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                   const int32_t* seq_lens, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                   int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t d,
+                   int64_t num_pages, int64_t page_size, int64_t max_pages_per_seq, int64_t num_splits,
+                   float scale, int mask_kind, int64_t window, cudaStream_t stream,
+                   const attn_fwd_options* opts);
+/* Workspace bytes attn_decode needs for num_splits (0 when num_splits == 1 or on invalid
+   sizes). */
+size_t attn_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t Nq, int64_t d, int64_t num_splits);
+/* Suggested num_splits for a step whose longest sequence has max_seq_len cached positions,
+   on the current device (one wave of work items, each split at least four 128-key tiles);
+   -1 on invalid sizes. Host-only. */
+int64_t attn_decode_num_splits(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t max_seq_len,
+                               int mask_kind, int64_t window);
+/* attn_debug_error for the decoding kernel's error word: ATTN_ERR_TIMEOUT for a wait
+   that gave up, ATTN_ERR_INVALID_ARG for a bad sequence length or page-table entry. */
+int attn_decode_debug_error(cudaStream_t stream, int* device_code);
 
 #ifdef __cplusplus
 }

@@ -135,3 +135,63 @@ def test_backward_valid_arguments_reach_the_device_check(lib):
         pytest.skip("GPU present")
     assert call_bwd(lib) == 4
     assert call_bwd(lib, d=128, mask=2, window=10 ** 9) == 4
+
+
+# ------------------------------------------------------------------ decoding
+KC, VC, BT, SL, DOUT, DLSE, DWS = (0x10000000000 * (i + 12) for i in range(7))
+
+
+def call_dec(lib, q=Q, kc=KC, vc=VC, bt=BT, sl=SL, o=DOUT, l=DLSE, ws=DWS, ws_bytes=None, B=2, Hq=8, Hkv=2, Nq=1,
+             d=128, num_pages=64, page_size=16, max_pages=32, splits=4, scale=0.088, mask=1, window=0):
+    if ws_bytes is None:
+        ws_bytes = lib.attn_decode_workspace_bytes(B, Hq, Nq, d, splits)
+    return lib.attn_decode(q, kc, vc, bt, sl, o, l, ws, ws_bytes, B, Hq, Hkv, Nq, d, num_pages, page_size,
+                           max_pages, splits, scale, mask, window, None)
+
+
+def test_decode_workspace_bytes(lib):
+    rows = 2 * 8 * 3
+    assert lib.attn_decode_workspace_bytes(2, 8, 3, 128, 1) == 0
+    lse_part = -(-(rows * 5 * 4) // 256) * 256
+    assert lib.attn_decode_workspace_bytes(2, 8, 3, 128, 5) == lse_part + rows * 5 * 128 * 4
+    assert lib.attn_decode_workspace_bytes(2, 8, 3, 96, 5) == 0
+    assert lib.attn_decode_workspace_bytes(0, 8, 3, 64, 5) == 0
+    assert lib.attn_decode_workspace_bytes(1, 8, 3, 64, 0) == 0
+
+
+def test_decode_num_splits_without_a_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present: the count depends on its SM count")
+    # 148 SMs assumed: one wave of items, at least four 128-key tiles per split
+    assert lib.attn_decode_num_splits(1, 64, 8, 1, 131072, 1, 0) == 148 // 8
+    assert lib.attn_decode_num_splits(32, 32, 8, 1, 131072, 1, 0) == 1
+    assert lib.attn_decode_num_splits(1, 64, 8, 1, 1000, 1, 0) == 2      # (8 + 1) // 4 tiles limit
+    assert lib.attn_decode_num_splits(1, 32, 8, 1, 131072, 2, 4096) == (4096 // 128 + 1) // 4
+    assert lib.attn_decode_num_splits(1, 64, 8, 1, 0, 1, 0) == -1
+    assert lib.attn_decode_num_splits(1, 6, 4, 1, 100, 1, 0) == -1
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(kc=None), 1), (dict(vc=None), 1), (dict(bt=None), 1), (dict(sl=None), 1),
+    (dict(o=None), 1), (dict(l=None), 1), (dict(ws=None), 1), (dict(ws_bytes=16), 1),
+    (dict(B=0), 1), (dict(Hq=6, Hkv=4), 1), (dict(Nq=0), 1), (dict(num_pages=0), 1), (dict(max_pages=0), 1),
+    (dict(splits=0), 1), (dict(splits=5000), 1), (dict(mask=3), 1), (dict(mask=2, window=0), 1),
+    (dict(scale=0.0), 1), (dict(scale=float("nan")), 1),
+    (dict(d=96), 2), (dict(page_size=8), 2), (dict(page_size=48), 2), (dict(page_size=512), 2),
+    (dict(q=Q + 8), 3), (dict(kc=KC + 8), 3), (dict(vc=VC + 4), 3), (dict(o=DOUT + 2), 3), (dict(l=DLSE + 2), 3),
+    (dict(bt=BT + 2), 3), (dict(sl=SL + 1), 3), (dict(ws=DWS + 4), 3),
+    (dict(o=Q), 1), (dict(l=KC + 64), 1), (dict(ws=BT), 1), (dict(o=SL), 1), (dict(l=DOUT + 256), 1),
+    (dict(ws=DLSE), 1),
+])
+def test_decode_invalid_arguments_rejected_before_launch(lib, kw, status):
+    assert call_dec(lib, **kw) == status
+
+
+def test_decode_valid_arguments_reach_the_device_check(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    assert call_dec(lib) == 4
+    assert call_dec(lib, splits=1, ws=None, ws_bytes=0) == 4     # one split needs no workspace
+    assert call_dec(lib, Nq=40, d=64, page_size=256, mask=2, window=5) == 4
