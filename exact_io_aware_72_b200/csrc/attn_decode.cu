@@ -227,12 +227,14 @@ extern "C" int attn_decode_ex(const void* q, const void* k_cache, const void* v_
       return ATTN_ERR_CUDA;
   }
   for (int kv = 0; kv < 2; ++kv) {
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(page_size),
+    // 4-D view of a cache: (64 columns, page rows, d/64 column halves, page x KV head); a V box
+    // brings both halves of a page's rows, half after half, a K box one half.
+    cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(page_size), static_cast<cuuint64_t>(d / 64),
                           static_cast<cuuint64_t>(num_pages * Hkv)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(page_size * d * 2)};
-    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows_per_load), 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    if (enc(kv ? &p.tm_v : &p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv ? v_cache : k_cache),
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(d * 2), 128, static_cast<cuuint64_t>(page_size * d * 2)};
+    cuuint32_t box[4] = {64, static_cast<cuuint32_t>(rows_per_load), kv ? static_cast<cuuint32_t>(d / 64) : 1u, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (enc(kv ? &p.tm_v : &p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(kv ? v_cache : k_cache),
             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return ATTN_ERR_CUDA;

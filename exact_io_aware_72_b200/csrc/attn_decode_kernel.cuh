@@ -72,7 +72,7 @@ constexpr int kDErrPage = 2 << 20;     // a page-table entry the step needs is o
 
 struct DecParams {
   CUtensorMap tm_q;       // [1, B*Hq*Nq, d] bf16, box 64 x rows_chunk, 128-byte swizzle
-  CUtensorMap tm_k;       // [num_pages*Hkv, page_size, d] bf16, box 64 x rows_per_load x 1
+  CUtensorMap tm_k;       // [num_pages*Hkv][d/64][page_size][64] view, box 64 x rows_per_load x d/64 x 1
   CUtensorMap tm_v;
   const int* block_table; // [B, max_pages]
   const int* seq_lens;    // [B]
@@ -195,6 +195,17 @@ struct DecWaiter {
   }
 };
 
+// 4-D tiled load global -> shared (one page box: both 64-column halves of
+// rows_per_load rows), completing its bytes on the mbarrier.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y, int z,
+                                            int w, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ float dec_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -230,19 +241,24 @@ __device__ __forceinline__ void dec_loader(const DecParams& p, uint32_t sbase, c
     const DecItem it = dec_item(p, idx);
     if (it.t1 < it.t0) continue;
     const int* trow = p.block_table + static_cast<size_t>(it.b) * p.max_pages;
-    // Physical page of this lane's box in tile t, or -1 when the box holds no
-    // position of [lo_pos, L) (then nothing is loaded and the table entry is
-    // not read).
-    auto box_page = [&](int t) -> int {
-      if (lane >= p.loads_per_tile) return -1;
+    // Page-table entry of this lane's box in tile t, or -1 when the box holds
+    // no position of [lo_pos, L) (then nothing is loaded and the table entry
+    // is not read).  The entries are read two tiles ahead and checked only
+    // when used, so the table's load latency stays off the issue path.
+    auto box_entry = [&](int t) -> int {
+      if (t > it.t1 || lane >= p.loads_per_tile) return -1;
       const int pos0 = t * kKeys + lane * p.rows_per_load;
       if (pos0 >= it.L || pos0 + p.rows_per_load <= it.lo_pos) return -1;
-      int page = __ldg(trow + pos0 / p.page_size);
-      if (page < 0 || page >= p.num_pages) {
+      return __ldg(trow + pos0 / p.page_size);
+    };
+    auto checked = [&](int t, int entry) -> int {
+      const int pos0 = t * kKeys + lane * p.rows_per_load;
+      if (lane >= p.loads_per_tile || pos0 >= it.L || pos0 + p.rows_per_load <= it.lo_pos) return -1;
+      if (entry < 0 || entry >= p.num_pages) {
         atomicCAS(p.err, 0, kDErrPage | (it.b & 0xFFFFF));
-        page = 0;  // stand-in inside the pool; the step's result is then undefined
+        return 0;  // stand-in inside the pool; the step's result is then undefined
       }
-      return page;
+      return entry;
     };
     auto issue = [&](int t, int kv, int page) -> bool {
       const uint32_t slot = kv_n % L::kStages;
@@ -257,18 +273,28 @@ __device__ __forceinline__ void dec_loader(const DecParams& p, uint32_t sbase, c
       if (page >= 0) {
         const int y = (t * kKeys + lane * p.rows_per_load) % p.page_size;  // 0 unless pages exceed a tile
         const int z = page * p.Hkv + it.hkv;
-        const CUtensorMap* map = kv ? &p.tm_v : &p.tm_k;
-        const uint32_t dst = sbase + L::kRingOff + slot * L::kTileBytes + lane * p.rows_per_load * 128;
+        const uint32_t tile = sbase + L::kRingOff + slot * L::kTileBytes;
+        if (kv) {
+          // V: one box per page, both column halves, stored half after half
+          // ([half][R rows][128 B], the page's block of the tile).
+          tma_load_4d(tile + lane * p.rows_per_load * 128 * L::kChunks, &p.tm_v, bar(L::kKVFull + slot), 0, y, 0, z,
+                      pol);
+        } else {
+          // K: one box per page and column half into the [half][128 rows]
+          // tile that a single N = 128 product reads.
 #pragma unroll
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(dst + c * L::kChunkBytes, map, bar(L::kKVFull + slot), c * 64, y, z, pol);
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_4d(tile + c * L::kChunkBytes + lane * p.rows_per_load * 128, &p.tm_k, bar(L::kKVFull + slot), 0,
+                        y, c, z, pol);
+        }
       }
       ++kv_n;
       return true;
     };
-    int pg = box_page(it.t0);
+    int e0 = box_entry(it.t0), e1 = box_entry(it.t0 + 1);
     for (int t = it.t0; t <= it.t1; ++t) {
-      const int pg_next = (t < it.t1) ? box_page(t + 1) : -1;  // table entries one tile ahead
+      const int e2 = box_entry(t + 2);
+      const int pg = checked(t, e0);
       if (!issue(t, 0, pg) || !issue(t, 1, pg)) {
         ok = false;
         break;
@@ -292,7 +318,8 @@ __device__ __forceinline__ void dec_loader(const DecParams& p, uint32_t sbase, c
         __syncwarp();
         ++q_n;
       }
-      pg = pg_next;
+      e0 = e1;
+      e1 = e2;
     }
   }
   // Drain: every copy this warp started must land before the CTA exits.
@@ -309,7 +336,9 @@ __device__ __forceinline__ void dec_loader(const DecParams& p, uint32_t sbase, c
 }
 
 // MMA warp: per item S_0, then for each tile j: S_{j+1} (look-ahead into the
-// other S buffer) and O += P_j V_j once the softmax has published P_j.
+// other S buffer) and O += P_j V_j once the softmax has published P_j.  S_j is
+// always issued after P V of tile j-2 (in-order completion then makes "S_j
+// done" imply "P V_{j-2} done"), whichever of S_{j+1} and P V_j goes first.
 template <int D>
 __device__ __forceinline__ void dec_mma(const DecParams& p, uint32_t sbase, uint32_t tmem, const DecWaiter& w) {
   using L = DecSmem<D>;
@@ -317,8 +346,13 @@ __device__ __forceinline__ void dec_mma(const DecParams& p, uint32_t sbase, uint
   constexpr uint32_t idesc_s = idesc_bf16_f32(kLanes, kKeys, false);
   constexpr uint32_t idesc_o = idesc_bf16_f32(kLanes, D, true);
   const uint64_t q_desc = smem_desc_sw128(sbase + L::kQOff, 16, 1024);
+  // A K tile is [half][128 rows][128 B]; a V tile is 128 / R page blocks of
+  // [half][R rows][128 B] (R = rows_per_load), which for one column half or
+  // R = 128 is the same thing.
+  const int R = p.rows_per_load;
+  const uint32_t box_bytes = static_cast<uint32_t>(R) * 128u * L::kChunks;
   const uint64_t k_desc0 = smem_desc_sw128(sbase + L::kRingOff, 16, 1024);
-  const uint64_t v_desc0 = smem_desc_sw128(sbase + L::kRingOff, L::kChunkBytes, 1024);
+  const uint64_t v_desc0 = smem_desc_sw128(sbase + L::kRingOff, static_cast<uint32_t>(R) * 128u, 1024);
   const uint32_t o_tmem = tmem + L::kOCol;
   const int code = kDRoleMma << 8;
   uint32_t g = 0, q_n = 0, items = 0;
@@ -348,9 +382,19 @@ __device__ __forceinline__ void dec_mma(const DecParams& p, uint32_t sbase, uint
     };
     if (!issue_s(0)) break;
     for (int j = 0; j < n; ++j) {
-      if (j + 1 < n && !issue_s(j + 1)) {
-        ok = false;
-        break;
+      // S of the next tile goes first when its K has landed (the softmax can
+      // then start that tile as soon as it finishes this one); otherwise this
+      // tile's P V goes first, so its V slot is not held while K is awaited.
+      bool s_next_done = j + 1 >= n;
+      if (!s_next_done) {
+        const uint32_t kidx = 2 * (g + j + 1);
+        if (__all_sync(0xffffffffu, mbar_try_wait(bar(L::kKVFull + kidx % L::kStages), (kidx / L::kStages) & 1))) {
+          if (!issue_s(j + 1)) {
+            ok = false;
+            break;
+          }
+          s_next_done = true;
+        }
       }
       const uint32_t gi = g + j, vidx = 2 * gi + 1, vslot = vidx % L::kStages;
       if (!w.wait_warp(bar(L::kPFull + (gi & 1)), (gi >> 1) & 1, code | (L::kPFull + (gi & 1))) ||
@@ -363,11 +407,18 @@ __device__ __forceinline__ void dec_mma(const DecParams& p, uint32_t sbase, uint
       const uint32_t p_tmem = tmem + L::kPCol + 64 * (gi & 1);
       const uint64_t vd = v_desc0 + ((vslot * L::kTileBytes) >> 4);
 #pragma unroll
-      for (int kk = 0; kk < kKeys / 16; ++kk)
-        mma_bf16_ts_elect(o_tmem, p_tmem + kk * 8, vd + ((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < kKeys / 16; ++kk) {
+        // keys 16 kk .. 16 kk + 15: box block (16 kk) / R, rows from (16 kk) % R
+        const uint32_t voff = ((16 * kk) / R * box_bytes + ((16 * kk) % R) * 128) >> 4;
+        mma_bf16_ts_elect(o_tmem, p_tmem + kk * 8, vd + voff, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+      }
       tc_commit_elect(bar(L::kPVDone));
       if (j == n - 1) tc_commit_elect(bar(L::kODone));
       tc_commit_elect(bar(L::kKVEmpty + vslot));
+      if (!s_next_done && !issue_s(j + 1)) {
+        ok = false;
+        break;
+      }
     }
     g += n;
     ++items;
@@ -547,13 +598,16 @@ __device__ __forceinline__ void dec_softmax(const DecParams& p, uint32_t sbase, 
         for (int e = tid; e < nrows * 8 * L::kChunks; e += kLanes) {
           const int rr = e / (8 * L::kChunks), rem = e - rr * (8 * L::kChunks);
           const int row = rr < z0 ? rr : z1 + (rr - z0);
-          vt[((rem >> 3) * L::kChunkBytes + row * 128) / 16 + (rem & 7)] = make_uint4(0u, 0u, 0u, 0u);
+          const int R = p.rows_per_load;
+          vt[((row / R) * R * 128 * L::kChunks + (rem >> 3) * R * 128 + (row % R) * 128) / 16 + (rem & 7)] =
+              make_uint4(0u, 0u, 0u, 0u);
         }
         fence_proxy_async_smem();
       }
       tmem_store_wait();
       tc_fence_before_sync();
-      mbar_arrive(bar(L::kPFull + (gi & 1)));
+      __syncwarp();
+      if ((tid & 31) == 0) mbar_arrive(bar(L::kPFull + (gi & 1)));
     }
     if (!ok) break;
 
@@ -653,7 +707,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(L::kSFull + b), 1);
-      mbar_init(bar(L::kPFull + b), kLanes);  // every softmax thread arrives
+      mbar_init(bar(L::kPFull + b), 4);       // one arrival per softmax warp
     }
     mbar_init(bar(L::kPVDone), 1);
     mbar_init(bar(L::kODone), 1);
