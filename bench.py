@@ -476,7 +476,7 @@ def run_decode(args, w):
     out = torch.empty_like(inp["q"])
     lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=device)
     ws_bytes = decode_workspace_bytes(w.B, w.Hq, w.Nq, w.d, splits)
-    ws = torch.empty(max(ws_bytes // 4, 1), dtype=torch.float32, device=device)
+    ws = torch.zeros(ws_bytes // 4, dtype=torch.float32, device=device)  # counter must start at zero
     stream = torch.cuda.current_stream(device)
     nbytes = decode_bytes(w, lens)
 

@@ -224,8 +224,9 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
     block_table: [B,max_pages] int32; seq_lens: [B] int32 cached positions per
     sequence (new tokens included).  ``max_seq_len`` (a host-side upper bound
     of seq_lens, default max_pages*page_size) only picks the default
-    ``num_splits``.  The fp32 workspace for the splits' partial results is
-    allocated here when not given.
+    ``num_splits``.  The workspace (work counter and the splits' partial
+    results) is allocated here, zero-filled, when not given; a caller's own
+    workspace must start zeroed and is left with its counter at zero.
     """
     lib = load_library()
     _check(q, "q", torch.bfloat16, 4)
@@ -254,13 +255,12 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
     _check(out, "out", torch.bfloat16, 4)
     _check(lse, "lse", torch.float32, 3)
     ws_bytes = decode_workspace_bytes(B, Hq, Nq, d, num_splits)
-    if workspace is None and ws_bytes > 0:
-        workspace = torch.empty(ws_bytes // 4, dtype=torch.float32, device=q.device)
-    ws_ptr, ws_len = 0, 0
-    if workspace is not None:
-        if not (workspace.is_cuda and workspace.is_contiguous()):
-            raise ValueError("workspace must be a contiguous CUDA tensor")
-        ws_ptr, ws_len = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    if workspace is None:
+        # zero-filled: its first 256 bytes are the work counter, which each call leaves at zero
+        workspace = torch.zeros(ws_bytes // 4, dtype=torch.float32, device=q.device)
+    if not (workspace.is_cuda and workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_ptr, ws_len = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     opts = FwdOptions(int(wait_timeout_ns), 0, int(grid_ctas))

@@ -102,9 +102,13 @@ int warps_per_copy(int rows_chunk) { return rows_chunk <= 32 ? 1 : (rows_chunk <
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Workspace: 256 bytes of work-item counters (zero between calls), then with
+// more than one split the partial log-sum-exps and the partial outputs.
+constexpr size_t kSchedBytes = 256;
 size_t workspace_bytes(int64_t rows, int64_t d, int64_t splits) {
-  if (splits <= 1) return 0;
-  return align_up(static_cast<size_t>(rows) * splits * 4, 256) + static_cast<size_t>(rows) * splits * d * 4;
+  if (splits <= 1) return kSchedBytes;
+  return kSchedBytes + align_up(static_cast<size_t>(rows) * splits * 4, 256) +
+         static_cast<size_t>(rows) * splits * d * 4;
 }
 
 template <int D, int WC>
@@ -149,13 +153,17 @@ extern "C" int64_t attn_decode_num_splits(int64_t B, int64_t Hq, int64_t Hkv, in
   const int64_t rows_total = (Hq / Hkv) * Nq;
   const int64_t chunks = (rows_total + kLanes - 1) / kLanes;
   const int64_t units = B * Hkv * chunks;
-  if (units >= sms) return 1;
   int64_t keys = max_seq_len;
   if (mask_kind == ATTN_MASK_SLIDING_WINDOW) keys = std::min<int64_t>(keys, window + Nq - 1);
   const int64_t tiles = (keys + kKeys - 1) / kKeys + 1;
-  // One wave of items, each split at least four tiles long.
-  const int64_t s = std::min<int64_t>(sms / units, std::max<int64_t>(1, tiles / 4));
-  return std::max<int64_t>(1, std::min<int64_t>(s, kMaxSplits));
+  // A batch smaller than the SM count is split into one wave of items (each
+  // SM streams one item).  A larger batch takes several waves from the shared
+  // counter; there no item is longer than kMaxItemTiles tiles, so the SMs
+  // finish together even when sequence lengths differ.  Each split keeps at
+  // least four tiles.
+  constexpr int64_t kMaxItemTiles = 64;
+  const int64_t s = units < sms ? sms / units : (tiles + kMaxItemTiles - 1) / kMaxItemTiles;
+  return std::max<int64_t>(1, std::min<int64_t>({s, std::max<int64_t>(1, tiles / 4), kMaxSplits}));
 }
 
 extern "C" int attn_decode_ex(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
@@ -186,9 +194,9 @@ extern "C" int attn_decode_ex(const void* q, const void* k_cache, const void* v_
   if (B * Hkv > lim / row_chunks || B * Hkv * row_chunks > lim / num_splits) return ATTN_ERR_INVALID_ARG;
   const int64_t items = B * Hkv * row_chunks * num_splits;
   const size_t ws_need = workspace_bytes(rows, d, num_splits);
-  if (ws_need > 0 && (!workspace || workspace_bytes_given < ws_need)) return ATTN_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes_given < ws_need) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
-      !aligned(block_table, 4) || !aligned(seq_lens, 4) || (ws_need > 0 && !aligned(workspace, 16)))
+      !aligned(block_table, 4) || !aligned(seq_lens, 4) || !aligned(workspace, 16))
     return ATTN_ERR_MISALIGNED;
 
   const size_t q_bytes = static_cast<size_t>(rows) * d * 2;
@@ -243,10 +251,11 @@ extern "C" int attn_decode_ex(const void* q, const void* k_cache, const void* v_
   p.seq_lens = seq_lens;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  if (ws_need > 0) {
-    p.part_lse = static_cast<float*>(workspace);
-    p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                        align_up(static_cast<size_t>(rows) * num_splits * 4, 256));
+  p.sched = static_cast<unsigned int*>(workspace);
+  if (num_splits > 1) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace) + kSchedBytes;
+    p.part_lse = reinterpret_cast<float*>(ws);
+    p.part_o = reinterpret_cast<float*>(ws + align_up(static_cast<size_t>(rows) * num_splits * 4, 256));
   }
   p.err = dev.err_word;
   p.B = static_cast<int>(B);

@@ -14,7 +14,9 @@
 // * Work item = (sequence b, KV head, chunk of the group's query rows, split
 //   s of the visible key range).  Splits spread one long sequence over many
 //   SMs; a second kernel merges the splits' partial results by their
-//   log-sum-exp.  Items are dealt round-robin to one persistent CTA per SM.
+//   log-sum-exp.  One persistent CTA per SM takes items from a shared
+//   counter as it finishes the previous one, so sequences of different
+//   lengths balance across SMs.
 // * The group's query rows (Hq/Hkv heads x Nq new tokens, at most 128) form
 //   the 128-lane M dimension of the tcgen05 MMAs.  With R rows the rows are
 //   replicated into 128 / (32 * WC) copies (WC = warps per copy = ceil(R/32)
@@ -63,6 +65,9 @@ constexpr float kDecLn2 = 0.6931471805599453f;
 // forward): P may then exceed 1 by up to 2^32, which bf16 P and fp32 sums and
 // accumulators carry without loss, and the final merge uses the same maxima.
 constexpr float kDecRescaleThreshold = 32.0f;
+// Work items are handed out by a counter in global memory; the loader fetches
+// them and passes each index to the other roles through this many slots.
+constexpr int kItemSlots = 4;
 
 enum : int { kDMaskFull = 0, kDMaskCausal = 1, kDMaskWindow = 2 };
 enum : int { kDRoleLoader = 1, kDRoleMma = 2, kDRoleSoftmax = 3 };
@@ -90,6 +95,7 @@ struct DecParams {
   int num_splits, num_items;
   float scale_log2;       // scale * log2(e)
   unsigned long long timeout_ns;
+  unsigned int* sched;    // [0] next work item, [1] CTAs finished; zero between launches
 };
 
 template <int D>
@@ -116,9 +122,12 @@ struct DecSmem {
   static constexpr int kOFree = kODone + 1;
   static constexpr int kEpi = kOFree + 1;             // softmax warps' own barrier
   static constexpr int kFin = kEpi + 1;
-  static constexpr int kNumBars = kFin + 1;
+  static constexpr int kItemFull = kFin + 1;          // x kItemSlots
+  static constexpr int kItemEmpty = kItemFull + kItemSlots;
+  static constexpr int kNumBars = kItemEmpty + kItemSlots;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr uint32_t kBytes = kMiscOff + 16;
+  static constexpr uint32_t kItemOff = kMiscOff + 16;  // kItemSlots work-item indices
+  static constexpr uint32_t kBytes = kItemOff + 4 * kItemSlots;
   static constexpr uint32_t kAlloc = kBytes + 1024;   // slack to align the base to 1024 B
   static constexpr uint32_t kSCol = 0;                // + 128 * buffer
   static constexpr uint32_t kPCol = 256;              // + 64 * buffer
@@ -217,12 +226,29 @@ __device__ __forceinline__ uint32_t dec_pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Next work item of this CTA for a consuming role (every lane of the warp
+// calls it): the index the loader published in the next slot, or -1 if the
+// CTA aborts.  One lane per warp frees the slot after the warp has read it.
+template <int D>
+__device__ __forceinline__ int dec_take_item(uint32_t sbase, const uint8_t* smem, const DecWaiter& w, uint32_t& k,
+                                             int code) {
+  using L = DecSmem<D>;
+  const uint32_t slot = k % kItemSlots;
+  const uint32_t full = sbase + L::kBarOff + 8u * (L::kItemFull + slot);
+  if (!w.wait_warp(full, (k / kItemSlots) & 1, code | (L::kItemFull + slot))) return -1;
+  const int idx = *reinterpret_cast<const volatile int*>(smem + L::kItemOff + 4 * slot);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(sbase + L::kBarOff + 8u * (L::kItemEmpty + slot));
+  ++k;
+  return idx;
+}
+
 // ------------------------------------------------------------ roles
 // Loader warp: for every tile of an item, K then V into the next ring slots.
 // Lane i < loads_per_tile copies the tile's rows [i*R, i*R + R) (R =
 // rows_per_load) from the page holding them; lane 0 sets the expected bytes.
 template <int D, int WC>
-__device__ __forceinline__ void dec_loader(const DecParams& p, uint32_t sbase, const DecWaiter& w) {
+__device__ __forceinline__ void dec_loader(const DecParams& p, uint32_t sbase, uint8_t* smem, const DecWaiter& w) {
   using L = DecSmem<D>;
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
   const int lane = threadIdx.x & 31;
@@ -235,9 +261,26 @@ __device__ __forceinline__ void dec_loader(const DecParams& p, uint32_t sbase, c
   const int code = kDRoleLoader << 8;
   constexpr int kCopies = 4 / WC;   // replicas of the item's query rows
   constexpr int kRpc = 32 * WC;     // TMEM lanes per replica
-  uint32_t kv_n = 0, q_n = 0;
+  uint32_t kv_n = 0, q_n = 0, k_item = 0;
   bool ok = true;
-  for (int idx = blockIdx.x; ok && idx < p.num_items; idx += gridDim.x) {
+  // Work items come from the shared counter, one ahead of use so that the
+  // atomic's latency overlaps the current item; each index is published to
+  // the other roles before the item's loads start.
+  int next = 0;
+  if (lane == 0) next = static_cast<int>(atomicAdd(p.sched, 1u));
+  while (ok) {
+    const uint32_t slot_i = k_item % kItemSlots;
+    if (k_item >= (uint32_t)kItemSlots &&
+        !w.wait_warp(bar(L::kItemEmpty + slot_i), ((k_item / kItemSlots) - 1) & 1, code | (L::kItemEmpty + slot_i)))
+      break;
+    const int idx = __shfl_sync(0xffffffffu, next, 0);
+    if (lane == 0) {
+      *reinterpret_cast<volatile int*>(smem + L::kItemOff + 4 * slot_i) = idx < p.num_items ? idx : -2;
+      mbar_arrive(bar(L::kItemFull + slot_i));
+    }
+    ++k_item;
+    if (idx >= p.num_items) break;
+    if (lane == 0) next = static_cast<int>(atomicAdd(p.sched, 1u));
     const DecItem it = dec_item(p, idx);
     if (it.t1 < it.t0) continue;
     const int* trow = p.block_table + static_cast<size_t>(it.b) * p.max_pages;
@@ -340,7 +383,8 @@ __device__ __forceinline__ void dec_loader(const DecParams& p, uint32_t sbase, c
 // always issued after P V of tile j-2 (in-order completion then makes "S_j
 // done" imply "P V_{j-2} done"), whichever of S_{j+1} and P V_j goes first.
 template <int D>
-__device__ __forceinline__ void dec_mma(const DecParams& p, uint32_t sbase, uint32_t tmem, const DecWaiter& w) {
+__device__ __forceinline__ void dec_mma(const DecParams& p, uint32_t sbase, const uint8_t* smem, uint32_t tmem,
+                                        const DecWaiter& w) {
   using L = DecSmem<D>;
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
   constexpr uint32_t idesc_s = idesc_bf16_f32(kLanes, kKeys, false);
@@ -355,9 +399,11 @@ __device__ __forceinline__ void dec_mma(const DecParams& p, uint32_t sbase, uint
   const uint64_t v_desc0 = smem_desc_sw128(sbase + L::kRingOff, static_cast<uint32_t>(R) * 128u, 1024);
   const uint32_t o_tmem = tmem + L::kOCol;
   const int code = kDRoleMma << 8;
-  uint32_t g = 0, q_n = 0, items = 0;
+  uint32_t g = 0, q_n = 0, items = 0, k_item = 0;
   bool ok = true;
-  for (int idx = blockIdx.x; ok && idx < p.num_items; idx += gridDim.x) {
+  while (ok) {
+    const int idx = dec_take_item<D>(sbase, smem, w, k_item, code);
+    if (idx < 0) break;
     const DecItem it = dec_item(p, idx);
     if (it.t1 < it.t0) continue;
     const int n = it.t1 - it.t0 + 1;
@@ -463,7 +509,7 @@ __device__ __forceinline__ void dec_softmax(const DecParams& p, uint32_t sbase, 
     tmem_store_wait();
   }
 
-  uint32_t g = 0, items = 0, epi = 0;
+  uint32_t g = 0, items = 0, epi = 0, k_item = 0;
   bool ok = true;
   // Barrier of the 128 softmax threads (bounded, unlike bar.sync).
   auto epi_sync = [&]() -> bool {
@@ -473,7 +519,9 @@ __device__ __forceinline__ void dec_softmax(const DecParams& p, uint32_t sbase, 
     return __all_sync(0xffffffffu, got);
   };
 
-  for (int idx = blockIdx.x; ok && idx < p.num_items; idx += gridDim.x) {
+  while (ok) {
+    const int idx = dec_take_item<D>(sbase, smem, w, k_item, code);
+    if (idx < 0) break;
     const DecItem it = dec_item(p, idx);
     const size_t grow0 = (static_cast<size_t>(it.b) * p.Hq + static_cast<size_t>(it.hkv) * p.group) * p.Nq + it.row0;
     if (it.t1 < it.t0) {
@@ -714,6 +762,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
     mbar_init(bar(L::kOFree), kLanes);
     mbar_init(bar(L::kEpi), kLanes);
     mbar_init(bar(L::kFin), 1);
+    for (int i = 0; i < kItemSlots; ++i) {
+      mbar_init(bar(L::kItemFull + i), 1);
+      mbar_init(bar(L::kItemEmpty + i), 5);  // the MMA warp and the four softmax warps
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -730,9 +782,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
   if (warp < 4) {
     dec_softmax<D, WC>(p, sbase, smem, tmem, w);
   } else if (warp == kDecLoaderWarp) {
-    dec_loader<D, WC>(p, sbase, w);
+    dec_loader<D, WC>(p, sbase, smem, w);
   } else {
-    dec_mma<D>(p, sbase, tmem, w);
+    dec_mma<D>(p, sbase, smem, tmem, w);
   }
 
   tc_fence_before_sync();
@@ -740,6 +792,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
   if (warp == kDecMmaWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, kDecTmemCols);
+  }
+  // The last CTA to finish puts the work counter back to zero for the next
+  // launch (every CTA has taken its last index by now).
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.sched, 0u);
+      atomicExch(p.sched + 1, 0u);
+    }
   }
 }
 

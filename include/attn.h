@@ -187,8 +187,11 @@ int attn_bwd_debug_error(cudaStream_t stream, int* device_code);
  *   out          device, bf16, [B, Hq, Nq, d], 16-byte aligned; fully overwritten
  *   lse          device, fp32, [B, Hq, Nq], 4-byte aligned; natural-log normaliser of each row
  *   workspace    device, 16-byte aligned, at least attn_decode_workspace_bytes(B, Hq, Nq, d,
- *                num_splits) bytes (none needed, may be NULL, when num_splits == 1); holds the
- *                splits' partial results until the merge launch of the same call has read them
+ *                num_splits) bytes, owned by the caller. Its first 256 bytes hold the counter
+ *                that hands work items to the SMs: they must be zero before the first call that
+ *                uses the workspace, and every call leaves them zero again. The rest holds the
+ *                splits' partial results until the merge launch of the same call has read them.
+ *                Calls that share a workspace must not run concurrently.
  *   Hq % Hkv == 0; query head h reads KV head h / (Hq / Hkv); d in {64, 128};
  *   page_size in {16, 32, 64, 128, 256}
  *   num_splits   1..4096: each sequence's visible key range is cut into this many parts
@@ -216,12 +219,13 @@ int attn_decode_ex(const void* q, const void* k_cache, const void* v_cache, cons
                    int64_t num_pages, int64_t page_size, int64_t max_pages_per_seq, int64_t num_splits,
                    float scale, int mask_kind, int64_t window, cudaStream_t stream,
                    const attn_fwd_options* opts);
-/* Workspace bytes attn_decode needs for num_splits (0 when num_splits == 1 or on invalid
-   sizes). */
+/* Workspace bytes attn_decode needs for num_splits (256 + the partial results when
+   num_splits > 1; 0 on invalid sizes). */
 size_t attn_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t Nq, int64_t d, int64_t num_splits);
 /* Suggested num_splits for a step whose longest sequence has max_seq_len cached positions,
-   on the current device (one wave of work items, each split at least four 128-key tiles);
-   -1 on invalid sizes. Host-only. */
+   on the current device: one wave of work items when B * Hkv (times the query-row chunks)
+   is below the SM count, otherwise splits of at most 64 128-key tiles; never a split
+   shorter than four tiles; -1 on invalid sizes. Host-only. */
 int64_t attn_decode_num_splits(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t max_seq_len,
                                int mask_kind, int64_t window);
 /* attn_debug_error for the decoding kernel's error word: ATTN_ERR_TIMEOUT for a wait

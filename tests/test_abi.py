@@ -151,9 +151,9 @@ def call_dec(lib, q=Q, kc=KC, vc=VC, bt=BT, sl=SL, o=DOUT, l=DLSE, ws=DWS, ws_by
 
 def test_decode_workspace_bytes(lib):
     rows = 2 * 8 * 3
-    assert lib.attn_decode_workspace_bytes(2, 8, 3, 128, 1) == 0
+    assert lib.attn_decode_workspace_bytes(2, 8, 3, 128, 1) == 256          # the work counter only
     lse_part = -(-(rows * 5 * 4) // 256) * 256
-    assert lib.attn_decode_workspace_bytes(2, 8, 3, 128, 5) == lse_part + rows * 5 * 128 * 4
+    assert lib.attn_decode_workspace_bytes(2, 8, 3, 128, 5) == 256 + lse_part + rows * 5 * 128 * 4
     assert lib.attn_decode_workspace_bytes(2, 8, 3, 96, 5) == 0
     assert lib.attn_decode_workspace_bytes(0, 8, 3, 64, 5) == 0
     assert lib.attn_decode_workspace_bytes(1, 8, 3, 64, 0) == 0
@@ -163,11 +163,15 @@ def test_decode_num_splits_without_a_device(lib):
     import torch
     if torch.cuda.is_available():
         pytest.skip("GPU present: the count depends on its SM count")
-    # 148 SMs assumed: one wave of items, at least four 128-key tiles per split
+    # 148 SMs assumed: one wave of items for small batches, else splits of at most 64 tiles;
+    # never fewer than 4 tiles per split
     assert lib.attn_decode_num_splits(1, 64, 8, 1, 131072, 1, 0) == 148 // 8
-    assert lib.attn_decode_num_splits(32, 32, 8, 1, 131072, 1, 0) == 1
-    assert lib.attn_decode_num_splits(1, 64, 8, 1, 1000, 1, 0) == 2      # (8 + 1) // 4 tiles limit
+    assert lib.attn_decode_num_splits(32, 32, 8, 1, 131072, 1, 0) == -(-(1024 + 1) // 64)
+    assert lib.attn_decode_num_splits(16, 32, 32, 1, 31004, 1, 0) == 4      # 244 tiles
+    assert lib.attn_decode_num_splits(1, 64, 8, 1, 1000, 1, 0) == 2         # (8 + 1) // 4 tiles limit
+    assert lib.attn_decode_num_splits(32, 32, 8, 1, 131072, 2, 4096) == 1   # 33-tile windows
     assert lib.attn_decode_num_splits(1, 32, 8, 1, 131072, 2, 4096) == (4096 // 128 + 1) // 4
+    assert lib.attn_decode_num_splits(8, 64, 8, 4, 31818, 1, 0) == 148 // 64          # one wave
     assert lib.attn_decode_num_splits(1, 64, 8, 1, 0, 1, 0) == -1
     assert lib.attn_decode_num_splits(1, 6, 4, 1, 100, 1, 0) == -1
 
@@ -175,6 +179,7 @@ def test_decode_num_splits_without_a_device(lib):
 @pytest.mark.parametrize("kw,status", [
     (dict(q=None), 1), (dict(kc=None), 1), (dict(vc=None), 1), (dict(bt=None), 1), (dict(sl=None), 1),
     (dict(o=None), 1), (dict(l=None), 1), (dict(ws=None), 1), (dict(ws_bytes=16), 1),
+    (dict(splits=1, ws=None), 1), (dict(splits=1, ws_bytes=128), 1),
     (dict(B=0), 1), (dict(Hq=6, Hkv=4), 1), (dict(Nq=0), 1), (dict(num_pages=0), 1), (dict(max_pages=0), 1),
     (dict(splits=0), 1), (dict(splits=5000), 1), (dict(mask=3), 1), (dict(mask=2, window=0), 1),
     (dict(scale=0.0), 1), (dict(scale=float("nan")), 1),
@@ -193,5 +198,5 @@ def test_decode_valid_arguments_reach_the_device_check(lib):
     if torch.cuda.is_available():
         pytest.skip("GPU present")
     assert call_dec(lib) == 4
-    assert call_dec(lib, splits=1, ws=None, ws_bytes=0) == 4     # one split needs no workspace
+    assert call_dec(lib, splits=1) == 4                          # one split: the counter only
     assert call_dec(lib, Nq=40, d=64, page_size=256, mask=2, window=5) == 4

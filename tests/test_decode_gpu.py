@@ -144,3 +144,20 @@ def test_workload_decode_swa(cuda_ok):
 
 def test_workload_decode_spec(cuda_ok):
     _check_workload("decode_spec", [0, 5])
+
+
+def test_shared_workspace_counter_returns_to_zero(cuda_ok):
+    from exact_io_aware_72_b200 import decode, decode_workspace_bytes
+    lens = [3000, 17, 900, 4000, 1]
+    inp = {k: v.cuda() for k, v in make_paged_kv(5, 8, 2, 1, 128, lens, 16, 8).items()}
+    ref = None
+    for splits, grid in ((1, 0), (3, 0), (3, 2), (1, 5)):
+        ws = torch.zeros(decode_workspace_bytes(5, 8, 1, 128, splits) // 4, device="cuda")
+        for _ in range(4):
+            out, lse = decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["block_table"], inp["seq_lens"],
+                              num_splits=splits, workspace=ws, grid_ctas=grid)
+            torch.cuda.synchronize()
+            assert int(ws[:64].view(torch.int32).abs().sum()) == 0     # the work counter is back at zero
+            if ref is None:
+                ref = oracle_for({k: v.cpu() for k, v in inp.items()}, "causal")
+            compare(to_np(out), to_np(lse), ref[0], ref[1], f"splits {splits} grid {grid}")
