@@ -75,6 +75,22 @@ def kernel_hash() -> str:
     return h.hexdigest()[:16]
 
 
+DECODE_KERNEL_SOURCES = ["exact_io_aware_72_b200/csrc/attn_decode_kernel.cuh", "exact_io_aware_72_b200/csrc/sm100_ptx.cuh"]
+# DRAM bytes per launch of the decoding kernel from one ncu capture, keyed by
+# workload and the hash of the decoding kernel's device sources.
+DECODE_NCU_TRAFFIC = {
+    ("decode_gqa", "f6e5801ad35ab3ab"): 537009152 + 4729856,   # profiles/attn_decode_gqa_ncu.md
+}
+
+
+def decode_kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in DECODE_KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -544,7 +560,8 @@ def run_decode(args, w):
                    "mask": w.mask, "window": w.window, "rolling_buffer": w.rolling, "num_splits": splits,
                    "bytes_per_step": nbytes, "l2": "KV cache larger than L2 (no flush)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
+                     "traffic": DECODE_NCU_TRAFFIC.get((w.name, decode_kernel_hash())),
+                     "peak_source": f"{peak_src} hbm_gbs",
                      "note": "achieved over the whole step (decoding kernel plus split merge)"},
         "gpu_launches": args.steps * (2 if splits > 1 else 1),
         "launch_ms": {"median": statistics.median(per_step_ms), "best": min(per_step_ms)},
