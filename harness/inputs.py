@@ -228,3 +228,22 @@ def make_decode_workload(w: DecodeWorkload, device="cpu", fill=None):
         keep = np.maximum(lens - w.Nq - w.window + 1, 0)
     return make_paged_kv(w.B, w.Hq, w.Hkv, w.Nq, w.d, lens, w.page_size, w.seed, device=device,
                          keep_from=keep, fill=fill)
+
+
+# ---------------------------------------------------------------- FP8 inputs
+def quantise_e4m3(t: torch.Tensor):
+    """Per-tensor E4M3 quantisation of a float tensor: scale = amax / 448 (the
+    largest finite E4M3 magnitude), codes = round-to-nearest E4M3 of t / scale
+    (torch's float8_e4m3fn cast).  Returns (uint8 codes, scale as a Python float)."""
+    amax = float(t.abs().max())
+    scale = amax / 448.0 if amax > 0 else 1.0
+    codes = (t.float() / scale).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes, scale
+
+
+def make_qkv_fp8(B, Hq, Hkv, N, d, seed, device="cpu", sharp=False):
+    """FP8 inputs: the bf16 recipe's fp32 draws (same generator, same order,
+    same sharp rows), each quantised per tensor with ``quantise_e4m3``.
+    Returns ((q8, sq), (k8, sk), (v8, sv))."""
+    q, k, v = make_qkv(B, Hq, Hkv, N, d, seed, device=device, sharp=sharp, dtype=torch.float32)
+    return quantise_e4m3(q), quantise_e4m3(k), quantise_e4m3(v)
