@@ -42,6 +42,8 @@ import torch  # noqa: E402
 from harness.inputs import DECODE_WORKLOADS, WORKLOADS, make_qkv, sample_rows  # noqa: E402
 
 METRIC = "attention fwd TFLOP/s (bf16, causal/window-adjusted) and % of B200 dense peak"
+FP8_METRIC = "attention fwd TFLOP/s (E4M3 inputs, causal/window-adjusted) and % of B200 dense fp8 peak"
+FP8_OVER_BF16 = 2.0  # nominal dense fp8 / bf16 tensor rate (4.5 / 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["exact_io_aware_72_b200/csrc/attn_fwd.cu", "exact_io_aware_72_b200/csrc/attn_fwd_kernel.cuh",
                   "exact_io_aware_72_b200/csrc/sm100_ptx.cuh"]
@@ -227,6 +229,25 @@ def cpu_baseline(w, q, k, v, target_s=15.0):
             "seconds": dt}
 
 
+def fp8_cpu_baseline(w, q8, k8, v8, sq, sk, sv):
+    """The fp64 FP8 oracle (decode, dequantise, forward definition) on 256
+    seeded query rows of one head, on the host cores."""
+    from threadpoolctl import threadpool_info
+    from oracle import attention_fp8 as O8
+    rows = sample_rows(w.N, w.window, w.seed + 100, count=min(w.N, 256))
+    g = w.Hq // w.Hkv
+    qh, kh, vh = (t[:1, :1].cpu().numpy() for t in (q8, k8[:, :1], v8[:, :1]))
+    t0 = time.perf_counter()
+    O8.attention_fp8(qh, kh, vh, sq, sk, sv, w.scale, w.mask_kind, w.window, rows=rows)
+    dt = time.perf_counter() - t0
+    from oracle import visible_count_per_row
+    flops = 4 * w.d * int(visible_count_per_row(w.N, w.mask_kind, w.window)[rows].sum())
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{len(rows)} seeded query rows of one head of the {w.name} workload (E4M3 decoded, "
+                      f"fp64 NumPy, scores materialised), {dt:.1f} s; group size {g}"}
+
+
 # ----------------------------------------------------------------- arms
 def run_reference(args, w):
     """The oracle as the reference arm: each step is a bounded sample of the
@@ -268,17 +289,27 @@ def run_ours(args, w):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    from exact_io_aware_72_b200 import fwd, fwd_host
+    from exact_io_aware_72_b200 import fwd, fwd_fp8, fwd_host
+    fp8 = args.dtype == "fp8"
 
     # Each rank runs its own shard of the global batch: B sequences seeded by rank.
-    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed + 1000 * rank, device=device, sharp=w.sharp)
-    out = torch.empty_like(q)
+    if fp8:
+        from harness.inputs import make_qkv_fp8
+        (q, sq), (k, sk), (v, sv) = make_qkv_fp8(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed + 1000 * rank, device=device,
+                                                 sharp=w.sharp)
+    else:
+        q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed + 1000 * rank, device=device, sharp=w.sharp)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=device)
     lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
     flops = workload_flops(w, w.B)
 
     def step():
-        fwd(q, k, v, scale=w.scale, mask=w.mask, window=w.window, out=out, lse=lse, stream=stream)
+        if fp8:
+            fwd_fp8(q, k, v, sq, sk, sv, scale=w.scale, mask=w.mask, window=w.window, out=out, lse=lse,
+                    stream=stream)
+        else:
+            fwd(q, k, v, scale=w.scale, mask=w.mask, window=w.window, out=out, lse=lse, stream=stream)
 
     clocks = ClockSampler(local)
     if rank == 0:
@@ -305,15 +336,29 @@ def run_ours(args, w):
 
     # End to end through the public host-buffer call: pinned q, k, v in, out and lse back.
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+
+    def e2e_step():
+        if fp8:
+            ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+            hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+            o, l = fwd_fp8(hq.to(device, non_blocking=True), hk.to(device, non_blocking=True),
+                           hv.to(device, non_blocking=True), sq, sk, sv, scale=w.scale, mask=w.mask,
+                           window=w.window)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(l, non_blocking=True)
+            torch.cuda.current_stream(device).synchronize()
+        else:
+            fwd_host(hq, hk, hv, device=device, scale=w.scale, mask=w.mask, window=w.window)
+
     for _ in range(2):
-        fwd_host(hq, hk, hv, device=device, scale=w.scale, mask=w.mask, window=w.window)
+        e2e_step()
     e2e_steps = max(3, min(args.steps, 20))
     torch.cuda.synchronize(device)
     barrier(world, device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        fwd_host(hq, hk, hv, device=device, scale=w.scale, mask=w.mask, window=w.window)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
@@ -324,13 +369,14 @@ def run_ours(args, w):
         peaks, peak_src = load_peaks()
         avg_launch_s = statistics.mean(per_launch_ms) / 1e3
         achieved = flops / avg_launch_s / 1e12
-        peak = float(peaks["bf16_tflops"])
+        peak = float(peaks["bf16_tflops"]) * (FP8_OVER_BF16 if fp8 else 1.0)
         value = world * flops * args.steps / (total_ms / 1e3) / 1e12
-        traffic = NCU_TRAFFIC.get((w.name, kernel_hash()))
+        traffic = None if fp8 else NCU_TRAFFIC.get((w.name, kernel_hash()))
         line = {
-            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "metric": FP8_METRIC if fp8 else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
+            "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
                        "mask": w.mask, "window": w.window, "sharp_rows": w.sharp,
                        "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"dp{world}",
@@ -338,8 +384,10 @@ def run_ours(args, w):
             "frac_of_peak": value / world / peak,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"{peak_src} bf16_tflops (burst)",
-                         "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak))},
+                         "peak_source": (f"{peak_src} bf16_tflops (burst) x {FP8_OVER_BF16} (nominal fp8/bf16)"
+                                         if fp8 else f"{peak_src} bf16_tflops (burst)"),
+                         "frac_of_sustained": achieved / (float(peaks.get("bf16_tflops_sustained", peak)) *
+                                                          (FP8_OVER_BF16 if fp8 else 1.0))},
             "gpu_launches": args.steps,
             "launch_ms": {"median": statistics.median(per_launch_ms), "best": min(per_launch_ms)},
             "clocks": clk,
@@ -347,8 +395,11 @@ def run_ours(args, w):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         }
         if not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(w, q, k, v, target_s=args.cpu_seconds)
-            line["cpu_baseline"].pop("seconds", None)
+            if fp8:
+                line["cpu_baseline"] = fp8_cpu_baseline(w, q, k, v, sq, sk, sv)
+            else:
+                line["cpu_baseline"] = cpu_baseline(w, q, k, v, target_s=args.cpu_seconds)
+                line["cpu_baseline"].pop("seconds", None)
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -595,6 +646,8 @@ def main():
     ap.add_argument("--pass", dest="which", choices=["fwd", "bwd", "decode"], default="fwd",
                     help="bwd: the backward pass; decode: a paged-KV decoding step (one GPU each)")
     ap.add_argument("--splits", type=int, default=0, help="decode: KV splits per sequence (0 = suggested)")
+    ap.add_argument("--dtype", choices=["bf16", "fp8"], default="bf16",
+                    help="forward inputs: bf16, or E4M3 codes with per-tensor scales")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

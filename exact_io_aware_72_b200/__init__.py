@@ -1,11 +1,13 @@
-"""Exact attention forward, backward and paged-KV decoding for NVIDIA B200 (sm_100a).
+"""Exact attention forward (bf16 and FP8 inputs), backward and paged-KV decoding
+for NVIDIA B200 (sm_100a).
 
-``fwd``, ``bwd`` and ``decode`` run the hand-written tcgen05/TMA kernels of
+``fwd``, ``fwd_fp8``, ``bwd`` and ``decode`` run the hand-written tcgen05/TMA kernels of
 ``libattn_b200.so`` through its C ABI (include/attn.h); there is no CPU or
 library fallback.
 """
 from .attn import (AttnError, MASKS, bwd, bwd_debug_error, debug_error, decode, decode_debug_error,  # noqa: F401
-                   decode_num_splits, decode_workspace_bytes, fwd, fwd_host, load_library, num_work_items)
+                   decode_num_splits, decode_workspace_bytes, fwd, fwd_fp8, fwd_host, load_library,
+                   num_work_items)
 
-__all__ = ["fwd", "fwd_host", "bwd", "bwd_debug_error", "decode", "decode_debug_error", "decode_num_splits",
+__all__ = ["fwd", "fwd_fp8", "fwd_host", "bwd", "bwd_debug_error", "decode", "decode_debug_error", "decode_num_splits",
            "decode_workspace_bytes", "debug_error", "load_library", "num_work_items", "AttnError", "MASKS"]

@@ -21,7 +21,7 @@ LIB_NAME = "libattn_b200.so"
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_status_string", "attn_debug_error", "attn_fwd_num_work_items",
            "attn_bwd", "attn_bwd_ex", "attn_bwd_workspace_bytes", "attn_bwd_debug_error",
            "attn_decode", "attn_decode_ex", "attn_decode_workspace_bytes", "attn_decode_num_splits",
-           "attn_decode_debug_error")
+           "attn_decode_debug_error", "attn_fwd_fp8", "attn_fwd_fp8_ex")
 
 _lib = None
 
@@ -56,6 +56,12 @@ def load_library():
     lib.attn_fwd.restype = ctypes.c_int
     lib.attn_fwd_ex.argtypes = fwd_args + [ctypes.POINTER(FwdOptions)]
     lib.attn_fwd_ex.restype = ctypes.c_int
+    f32 = ctypes.c_float
+    fp8_args = [vp, vp, vp, f32, f32, f32, vp, vp, i64, i64, i64, i64, i64, f32, ctypes.c_int, i64, vp]
+    lib.attn_fwd_fp8.argtypes = fp8_args
+    lib.attn_fwd_fp8.restype = ctypes.c_int
+    lib.attn_fwd_fp8_ex.argtypes = fp8_args + [ctypes.POINTER(FwdOptions)]
+    lib.attn_fwd_fp8_ex.restype = ctypes.c_int
     lib.attn_status_string.argtypes = [ctypes.c_int]
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_debug_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
@@ -132,6 +138,50 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float
                              ctypes.byref(opts))
     if st != 0:
         raise AttnError(st, "attn_fwd")
+    return out, lse
+
+
+def _codes(t: torch.Tensor, name: str) -> torch.Tensor:
+    if isinstance(t, torch.Tensor) and t.dtype == torch.float8_e4m3fn:
+        t = t.view(torch.uint8)
+    _check(t, name, torch.uint8, 4)
+    return t
+
+
+def fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_scale: float, k_scale: float, v_scale: float,
+            scale: Optional[float] = None, mask: str = "causal", window: Optional[int] = None,
+            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+            stream: Optional[torch.cuda.Stream] = None, wait_timeout_ns: int = 0, grid_ctas: int = 0
+            ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Exact attention forward of E4M3 inputs: q, k, v hold E4M3 codes (uint8 or
+    torch.float8_e4m3fn, [B,H,N,128]) whose values are code * q_scale (k_scale,
+    v_scale); returns (out bf16 [B,Hq,N,128], lse fp32 [B,Hq,N])."""
+    lib = load_library()
+    q, k, v = _codes(q, "q"), _codes(k, "k"), _codes(v, "v")
+    B, Hq, N, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if (Bk, Nk, dk) != (B, N, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("q, k, v shapes disagree")
+    if mask not in MASKS:
+        raise ValueError(f"mask must be one of {sorted(MASKS)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    opts = FwdOptions(int(wait_timeout_ns), 0, int(grid_ctas))
+    with torch.cuda.device(q.device):
+        st = lib.attn_fwd_fp8_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), float(q_scale), float(k_scale),
+                                 float(v_scale), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, d, float(scale),
+                                 MASKS[mask], int(window) if window is not None else 0,
+                                 ctypes.c_void_p(stream.cuda_stream), ctypes.byref(opts))
+    if st != 0:
+        raise AttnError(st, "attn_fwd_fp8")
     return out, lse
 
 

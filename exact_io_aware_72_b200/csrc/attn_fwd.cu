@@ -46,7 +46,6 @@ struct DeviceInfo {
   bool probed = false;
   bool supported = false;
   int sm_count = 0;
-  bool smem_set[2] = {false, false};  // d = 64, d = 128
   int* err_word = nullptr;
 };
 
@@ -75,9 +74,10 @@ int device_setup(int& dev, DeviceInfo& out_info) {
       if (cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SmemLayout<64>::kAlloc) != cudaSuccess ||
           cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               SmemLayout<128>::kAlloc) != cudaSuccess)
+                               SmemLayout<128>::kAlloc) != cudaSuccess ||
+          cudaFuncSetAttribute(attn_fwd_kernel<128, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SmemLayout<128, 1>::kAlloc) != cudaSuccess)
         return ATTN_ERR_CUDA;
-      info.smem_set[0] = info.smem_set[1] = true;
     }
     info.probed = true;
   }
@@ -127,14 +127,100 @@ int check_sizes(int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d, int ma
   return ATTN_OK;
 }
 
-CUresult encode_bhnd(EncodeTiledFn enc, CUtensorMap* map, const void* base, int64_t BH, int64_t N, int64_t d) {
+// [BH, N, d] tensor of eb-byte elements (2: bf16, 1: E4M3 codes), boxes of
+// 128 rows x 128 bytes with the 128-byte swizzle.
+CUresult encode_bhnd(EncodeTiledFn enc, CUtensorMap* map, const void* base, int64_t BH, int64_t N, int64_t d,
+                     int eb = 2) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(N * d * 2)};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kBlockM), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * eb), static_cast<cuuint64_t>(N * d * eb)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(kBlockM), 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return enc(map, eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+// Shared by the bf16 (eb = 2) and E4M3 (eb = 1) entry points: checks, tensor
+// maps and the launch.  score_scale multiplies q.k of the stored values
+// (softmax scale, times the q and k scales for E4M3); v_scale multiplies O.
+int fwd_launch(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t Hq,
+               int64_t Hkv, int64_t N, int64_t d, int eb, float score_scale, float v_scale, int mask_kind,
+               int64_t window, cudaStream_t stream, const attn_fwd_options* opts) {
+  if (!q || !k || !v || !out || !lse) return ATTN_ERR_INVALID_ARG;
+  Plan plan{};
+  int st = check_sizes(B, Hq, Hkv, N, d, mask_kind, window, plan);
+  if (st != ATTN_OK) return st;
+  if (eb == 1 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!std::isfinite(score_scale) || !(score_scale > 0.f) || !std::isfinite(v_scale) || !(v_scale > 0.f))
+    return ATTN_ERR_INVALID_ARG;
+  const size_t q_bytes = static_cast<size_t>(B * Hq * N * d) * eb;
+  const size_t kv_bytes = static_cast<size_t>(B * Hkv * N * d) * eb;
+  const size_t out_bytes = static_cast<size_t>(B * Hq * N * d) * 2;
+  const size_t lse_bytes = static_cast<size_t>(B * Hq * N) * 4;
+  if (overlaps(out, out_bytes, q, q_bytes) || overlaps(out, out_bytes, k, kv_bytes) ||
+      overlaps(out, out_bytes, v, kv_bytes) || overlaps(lse, lse_bytes, out, out_bytes) ||
+      overlaps(lse, lse_bytes, q, q_bytes) || overlaps(lse, lse_bytes, k, kv_bytes) ||
+      overlaps(lse, lse_bytes, v, kv_bytes))
+    return ATTN_ERR_INVALID_ARG;
+  auto mis16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
+  if (mis16(q) || mis16(k) || mis16(v) || mis16(out) || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return ATTN_ERR_MISALIGNED;
+
+  int dev = 0;
+  DeviceInfo info;
+  st = device_setup(dev, info);
+  if (st != ATTN_OK) return st;
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return ATTN_ERR_CUDA;
+
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (encode_bhnd(enc, &p.tm_q, q, B * Hq, N, d, eb) != CUDA_SUCCESS ||
+      encode_bhnd(enc, &p.tm_k, k, B * Hkv, N, d, eb) != CUDA_SUCCESS ||
+      encode_bhnd(enc, &p.tm_v, v, B * Hkv, N, d, eb) != CUDA_SUCCESS)
+    return ATTN_ERR_CUDA;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.err = info.err_word;
+  p.B = static_cast<int>(B);
+  p.Hq = static_cast<int>(Hq);
+  p.Hkv = static_cast<int>(Hkv);
+  p.N = static_cast<int>(N);
+  p.group = static_cast<int>(Hq / Hkv);
+  p.mask_kind = plan.mask_kind;
+  p.window = static_cast<int>(plan.mask_kind == ATTN_MASK_SLIDING_WINDOW ? plan.window : N);
+  p.scale_log2 = score_scale * 1.4426950408889634f;
+  p.v_scale = v_scale;
+  p.pair_heads = plan.pair_heads;
+  p.num_mblk = static_cast<int>(plan.num_mblk);
+  p.row_units = static_cast<int>(plan.row_units);
+  p.head_units = static_cast<int>(plan.head_units);
+  p.num_items = static_cast<int>(plan.num_items);
+  p.timeout_ns = (opts && opts->wait_timeout_ns) ? opts->wait_timeout_ns : kDefaultTimeoutNs;
+  p.inject_stall = (opts && opts->inject_stall) ? 1 : 0;
+  p.out_v8 = (reinterpret_cast<uintptr_t>(out) % 32 == 0) ? 1 : 0;
+
+  int grid = info.sm_count;
+  if (opts && opts->grid_ctas > 0) grid = opts->grid_ctas;
+  if (grid > plan.super_items) grid = static_cast<int>(plan.super_items);
+
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cudaError_t e;
+  if (eb == 1) {
+    cfg.dynamicSmemBytes = SmemLayout<128, 1>::kAlloc;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, 1>, p);
+  } else if (d == 128) {
+    cfg.dynamicSmemBytes = SmemLayout<128>::kAlloc;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128>, p);
+  } else {
+    cfg.dynamicSmemBytes = SmemLayout<64>::kAlloc;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<64>, p);
+  }
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 }  // namespace
@@ -163,74 +249,24 @@ int64_t attn_fwd_num_work_items(int64_t B, int64_t Hq, int64_t Hkv, int64_t N, i
 int attn_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t Hq,
                 int64_t Hkv, int64_t N, int64_t d, float scale, int mask_kind, int64_t window, cudaStream_t stream,
                 const attn_fwd_options* opts) {
-  if (!q || !k || !v || !out || !lse) return ATTN_ERR_INVALID_ARG;
-  Plan plan{};
-  int st = check_sizes(B, Hq, Hkv, N, d, mask_kind, window, plan);
-  if (st != ATTN_OK) return st;
-  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
-  const size_t q_bytes = static_cast<size_t>(B * Hq * N * d) * 2;
-  const size_t kv_bytes = static_cast<size_t>(B * Hkv * N * d) * 2;
-  const size_t lse_bytes = static_cast<size_t>(B * Hq * N) * 4;
-  if (overlaps(out, q_bytes, q, q_bytes) || overlaps(out, q_bytes, k, kv_bytes) ||
-      overlaps(out, q_bytes, v, kv_bytes) || overlaps(lse, lse_bytes, out, q_bytes) ||
-      overlaps(lse, lse_bytes, q, q_bytes) || overlaps(lse, lse_bytes, k, kv_bytes) ||
-      overlaps(lse, lse_bytes, v, kv_bytes))
+  return fwd_launch(q, k, v, out, lse, B, Hq, Hkv, N, d, 2, scale, 1.f, mask_kind, window, stream, opts);
+}
+
+int attn_fwd_fp8_ex(const void* q, const void* k, const void* v, float q_scale, float k_scale, float v_scale,
+                    void* out, float* lse, int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d, float scale,
+                    int mask_kind, int64_t window, cudaStream_t stream, const attn_fwd_options* opts) {
+  if (!std::isfinite(q_scale) || !(q_scale > 0.f) || !std::isfinite(k_scale) || !(k_scale > 0.f) ||
+      !std::isfinite(scale) || !(scale > 0.f))
     return ATTN_ERR_INVALID_ARG;
-  auto mis16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
-  if (mis16(q) || mis16(k) || mis16(v) || mis16(out) || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
-    return ATTN_ERR_MISALIGNED;
+  return fwd_launch(q, k, v, out, lse, B, Hq, Hkv, N, d, 1, scale * q_scale * k_scale, v_scale, mask_kind, window,
+                    stream, opts);
+}
 
-  int dev = 0;
-  DeviceInfo info;
-  st = device_setup(dev, info);
-  if (st != ATTN_OK) return st;
-  EncodeTiledFn enc = encode_tiled_fn();
-  if (!enc) return ATTN_ERR_CUDA;
-
-  FwdParams p;
-  std::memset(&p, 0, sizeof(p));
-  if (encode_bhnd(enc, &p.tm_q, q, B * Hq, N, d) != CUDA_SUCCESS ||
-      encode_bhnd(enc, &p.tm_k, k, B * Hkv, N, d) != CUDA_SUCCESS ||
-      encode_bhnd(enc, &p.tm_v, v, B * Hkv, N, d) != CUDA_SUCCESS)
-    return ATTN_ERR_CUDA;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
-  p.err = info.err_word;
-  p.B = static_cast<int>(B);
-  p.Hq = static_cast<int>(Hq);
-  p.Hkv = static_cast<int>(Hkv);
-  p.N = static_cast<int>(N);
-  p.group = static_cast<int>(Hq / Hkv);
-  p.mask_kind = plan.mask_kind;
-  p.window = static_cast<int>(plan.mask_kind == ATTN_MASK_SLIDING_WINDOW ? plan.window : N);
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.pair_heads = plan.pair_heads;
-  p.num_mblk = static_cast<int>(plan.num_mblk);
-  p.row_units = static_cast<int>(plan.row_units);
-  p.head_units = static_cast<int>(plan.head_units);
-  p.num_items = static_cast<int>(plan.num_items);
-  p.timeout_ns = (opts && opts->wait_timeout_ns) ? opts->wait_timeout_ns : kDefaultTimeoutNs;
-  p.inject_stall = (opts && opts->inject_stall) ? 1 : 0;
-  p.out_v8 = (reinterpret_cast<uintptr_t>(out) % 32 == 0) ? 1 : 0;
-
-  int grid = info.sm_count;
-  if (opts && opts->grid_ctas > 0) grid = opts->grid_ctas;
-  if (grid > plan.super_items) grid = static_cast<int>(plan.super_items);
-
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kThreads);
-  cfg.stream = stream;
-  cudaError_t e;
-  if (d == 128) {
-    cfg.dynamicSmemBytes = SmemLayout<128>::kAlloc;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128>, p);
-  } else {
-    cfg.dynamicSmemBytes = SmemLayout<64>::kAlloc;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<64>, p);
-  }
-  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+int attn_fwd_fp8(const void* q, const void* k, const void* v, float q_scale, float k_scale, float v_scale,
+                 void* out, float* lse, int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d, float scale,
+                 int mask_kind, int64_t window, cudaStream_t stream) {
+  return attn_fwd_fp8_ex(q, k, v, q_scale, k_scale, v_scale, out, lse, B, Hq, Hkv, N, d, scale, mask_kind, window,
+                         stream, nullptr);
 }
 
 int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t Hq,

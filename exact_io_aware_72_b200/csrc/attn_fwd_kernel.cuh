@@ -60,6 +60,13 @@ constexpr float kRescaleThreshold = 32.0f;
 // The factor is common to every p of a row, so O / l is unaffected and the
 // log-sum-exp (from the fp32 sum) subtracts it exactly.
 constexpr float kP16Bias = 0.0028150156f;  // log2(1 + 2^-9)
+// E4M3 P (FP8 inputs): p is stored times 2^8, so weights down to 2^-14 of
+// the row max stay normal E4M3 numbers; the running max then moves whenever a
+// row's max grows by more than half a power of two (P <= 2^8.5 < 448, the
+// largest E4M3 value).  The factor is common to the row: O / l is unaffected
+// and the log-sum-exp subtracts it.
+constexpr float kP8Bias = 8.0f;
+constexpr float kRescaleThresholdE4M3 = 0.5f;
 // 2^f on [-1/2, 1/2]: degree-3 polynomial with minimal maximum relative error
 // (Remez exchange; csrc/fit_exp2_poly.py), max relative error 7.5e-5, used
 // after Cody-Waite reduction x = n + f for kPolyPairs of every 16 column pairs
@@ -102,15 +109,18 @@ struct FwdParams {
   unsigned long long timeout_ns;
   int inject_stall;
   int out_v8;        // 1: out is 32-byte aligned, rows are written with 32-byte stores
+  float v_scale;     // FP8 inputs: the V tensor's scale, applied to O in the epilogue
 };
 
-template <int D>
+// EB = bytes per input element: 2 for bf16, 1 for E4M3 (head dim 128 only).
+template <int D, int EB = 2>
 struct SmemLayout {
-  static_assert(D == 64 || D == 128, "head dim");
-  static constexpr int kChunks = D / 64;                         // 128-byte column chunks
+  static_assert((EB == 2 && (D == 64 || D == 128)) || (EB == 1 && D == 128), "head dim and element size");
+  static constexpr int kChunks = D * EB / 128;                   // 128-byte column chunks
+  static constexpr int kChunkElems = 128 / EB;                   // elements in a 128-byte chunk row
   static constexpr uint32_t kChunkBytes = kBlockM * 128;         // 128 rows x 128 B
   static constexpr uint32_t kTileBytes = kChunks * kChunkBytes;  // one Q, K or V tile
-  static constexpr int kStages = (D == 128) ? 5 : 8;             // K/V ring slots
+  static constexpr int kStages = (kChunks == 2) ? 5 : 8;         // K/V ring slots
   static constexpr uint32_t kQOff = 0;
   static constexpr uint32_t kKVOff = 2 * kTileBytes;
   static constexpr uint32_t kBarOff = kKVOff + kStages * kTileBytes;
@@ -298,28 +308,30 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ------------------------------------------------------------ roles
 // L2 prefetch of the next work item's Q tiles and of its first two K/V tiles
 // (sched has already moved past the current item).
-template <int D>
+template <int D, int EB>
 __device__ __forceinline__ void prefetch_next_item(const FwdParams& p, Schedule sched) {
+  using L = SmemLayout<D, EB>;
   int hu, r;
   if (!sched.next(hu, r)) return;
   const WorkItem n = decode_item(p, hu, r);
 #pragma unroll
-  for (int c = 0; c < D / 64; ++c) {
+  for (int c = 0; c < L::kChunks; ++c) {
+    const int x = c * L::kChunkElems;
 #pragma unroll
     for (int t = 0; t < 2; ++t)
-      if (n.valid[t]) tma_prefetch_3d(&p.tm_q, c * 64, n.mblk[t] * kBlockM, n.b * p.Hq + n.head[t]);
+      if (n.valid[t]) tma_prefetch_3d(&p.tm_q, x, n.mblk[t] * kBlockM, n.b * p.Hq + n.head[t]);
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       if (n.lo_u + j > n.hi_u) break;
-      tma_prefetch_3d(&p.tm_k, c * 64, (n.lo_u + j) * kBlockN, n.b * p.Hkv + n.hkv);
-      tma_prefetch_3d(&p.tm_v, c * 64, (n.lo_u + j) * kBlockN, n.b * p.Hkv + n.hkv);
+      tma_prefetch_3d(&p.tm_k, x, (n.lo_u + j) * kBlockN, n.b * p.Hkv + n.hkv);
+      tma_prefetch_3d(&p.tm_v, x, (n.lo_u + j) * kBlockN, n.b * p.Hkv + n.hkv);
     }
   }
 }
 
-template <int D>
+template <int D, int EB>
 __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sbase, const Waiter& w) {
-  using L = SmemLayout<D>;
+  using L = SmemLayout<D, EB>;
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
   const uint64_t pol_kv = l2_policy_evict_last();
   const uint64_t pol_q = l2_policy_evict_first();
@@ -350,7 +362,7 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sbase
 #pragma unroll
         for (int c = 0; c < L::kChunks; ++c)
           tma_load_3d(sbase + L::kQOff + t * L::kTileBytes + c * L::kChunkBytes, &p.tm_q, bar(L::kQFull),
-                      c * 64, it.mblk[t] * kBlockM, it.b * p.Hq + it.head[t], pol_q);
+                      c * L::kChunkElems, it.mblk[t] * kBlockM, it.b * p.Hq + it.head[t], pol_q);
       }
       return true;
     };
@@ -359,7 +371,7 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sbase
     // item's loads do not wait on DRAM.
     const int pf_step = max(it.lo_u, it.hi_u - kPrefetchSteps);
     for (int j = it.lo_u; j <= it.hi_u && ok; ++j) {
-      if (j == pf_step) prefetch_next_item<D>(p, sched);
+      if (j == pf_step) prefetch_next_item<D, EB>(p, sched);
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
         const uint32_t slot = kv_n % L::kStages;
@@ -374,7 +386,7 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sbase
 #pragma unroll
         for (int c = 0; c < L::kChunks; ++c)
           tma_load_3d(sbase + L::kKVOff + slot * L::kTileBytes + c * L::kChunkBytes, map,
-                      bar(L::kKVFull + slot), c * 64, j * kBlockN, it.b * p.Hkv + it.hkv, pol_kv);
+                      bar(L::kKVFull + slot), c * L::kChunkElems, j * kBlockN, it.b * p.Hkv + it.hkv, pol_kv);
         ++kv_n;
         if (j == it.lo_u && kv == 1 && !load_q()) {
           ok = false;
@@ -401,13 +413,17 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sbase
 //   S_t  = Q_t K_j^T          (after that P V in issue order, since P aliases S)
 // and releases K_j / V_{j-1} / Q with commits; the other tile's warp does the
 // same, so each ring slot is freed after both warps' reads complete.
-template <int D>
+template <int D, int EB>
 __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tmem, const Waiter& w,
                                          int t) {
-  using L = SmemLayout<D>;
+  using L = SmemLayout<D, EB>;
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
-  constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false);
-  constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, true);
+  // bf16 inputs: kind::f16; E4M3 inputs: kind::f8f6f4.  Either way one
+  // product takes 32 bytes of K per row: 16 bf16 or 32 E4M3 elements.
+  constexpr uint32_t idesc_s =
+      EB == 2 ? idesc_bf16_f32(kBlockM, kBlockN, false) : idesc_e4m3_f32(kBlockM, kBlockN, false);
+  constexpr uint32_t idesc_o = EB == 2 ? idesc_bf16_f32(kBlockM, D, true) : idesc_e4m3_f32(kBlockM, D, true);
+  constexpr int kKeysPerPv = 32 / EB;  // keys per P V product
   const uint32_t s_tmem = tmem + (t ? L::kSCol1 : L::kSCol0);
   const uint32_t o_tmem = tmem + (t ? L::kOCol1 : L::kOCol0);
   // Descriptor bases: Q_t (K-major), ring slot 0 as K (K-major) and as V
@@ -456,9 +472,14 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
       tc_fence_after_sync();
       const uint64_t vd = v_desc0 + ((vslot * L::kTileBytes) >> 4);
 #pragma unroll
-      for (int kk = 0; kk < kBlockN / 16; ++kk) {
-        // 16 keys = two 8-row swizzle atoms = 2048 B further into the V tile.
-        mma_bf16_ts_elect(o_tmem, s_tmem + kk * 8, vd + ((kk * 2048) >> 4), idesc_o, (kk > 0 || !first_pv) ? 1u : 0u);
+      for (int kk = 0; kk < kBlockN / kKeysPerPv; ++kk) {
+        // Next keys: 16 (bf16) or 32 (E4M3) rows of 128 B further into the V
+        // tile; their P is the next 8 TMEM columns (32 bytes per row).
+        const uint64_t vk = vd + ((kk * kKeysPerPv * 128) >> 4);
+        if constexpr (EB == 2)
+          mma_bf16_ts_elect(o_tmem, s_tmem + kk * 8, vk, idesc_o, (kk > 0 || !first_pv) ? 1u : 0u);
+        else
+          mma_e4m3_ts_elect(o_tmem, s_tmem + kk * 8, vk, idesc_o, (kk > 0 || !first_pv) ? 1u : 0u);
       }
       first_pv = false;
       pend = false;
@@ -486,11 +507,14 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
       if (valid && j >= lo && j <= hi) {
         const uint64_t kd = k_desc0 + ((kslot * L::kTileBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          // K-major operands: 16 elements = 32 B inside a 128 B swizzled row,
-          // the next 64 columns 16 KB further.
+        for (int kk = 0; kk < D * EB / 32; ++kk) {
+          // K-major operands: 32 B of a 128 B swizzled row per product, the
+          // next 128-byte chunk of the rows 16 KB further.
           const uint32_t off = ((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4;
-          mma_bf16_ss_elect(s_tmem, q_desc + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
+          if constexpr (EB == 2)
+            mma_bf16_ss_elect(s_tmem, q_desc + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
+          else
+            mma_e4m3_ss_elect(s_tmem, q_desc + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
         }
         tc_commit_elect(bar(L::kSFull + t));
         pend = true;
@@ -518,10 +542,12 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
   w.drain(bar(L::kFin + t), 0, code | (L::kFin + t));
 }
 
-template <int D>
+template <int D, int EB>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tmem,
                                              const Waiter& w, int warp, int lane) {
-  using L = SmemLayout<D>;
+  using L = SmemLayout<D, EB>;
+  constexpr float kBias = EB == 2 ? kP16Bias : kP8Bias;
+  constexpr float kThreshold = EB == 2 ? kRescaleThreshold : kRescaleThresholdE4M3;
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
   const int t = warp >> 2;
   const int quarter = warp & 3;
@@ -590,7 +616,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
         for (int i = 8; i < 128; i += 2) mx[(i >> 1) & 7] = max3f(mx[(i >> 1) & 7], s[i], s[i + 1]);
         const float tile_max = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
         const float m_new = fmaxf(m_run, tile_max * c);
-        need = m_new > m_run + kRescaleThreshold;
+        need = m_new > m_run + kThreshold;
         if (need) {
           alpha = fast_exp2(m_run - m_new);
           m_run = m_new;
@@ -613,7 +639,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
         // dominated by one key returns that key's v); the log-sum-exp uses the
         // fp32 sum of p.
         const uint64_t c2 = f32x2_pack(c, c);
-        const uint64_t nb2 = f32x2_pack(neg_base + kP16Bias, neg_base + kP16Bias);
+        const uint64_t nb2 = f32x2_pack(neg_base + kBias, neg_base + kBias);
         const uint64_t magic2 = f32x2_pack(kRoundMagic, kRoundMagic);
         const uint64_t nmagic2 = f32x2_pack(-kRoundMagic, -kRoundMagic);
         const uint64_t neg1 = f32x2_pack(-1.f, -1.f);
@@ -622,7 +648,8 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
         uint64_t so2 = 0, sl2 = 0;  // (+0.f, +0.f)
 #pragma unroll
         for (int chunk = 0; chunk < 4; ++chunk) {
-          uint32_t pk[16];
+          uint32_t pk[EB == 2 ? 16 : 8];   // P columns: two bf16 or four E4M3 values each
+          float prev0 = 0.f, prev1 = 0.f;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int e = chunk * 32 + 2 * i;
@@ -648,13 +675,27 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
               p0 = fast_exp2(x0);
               p1 = fast_exp2(x1);
             }
-            pk[i] = __byte_perm(__float_as_uint(p0), __float_as_uint(p1), 0x7632);  // truncate to bf16x2
-            so2 = f32x2_add(so2, f32x2_pack(__uint_as_float(__float_as_uint(p0) & 0xffff0000u),
-                                            __uint_as_float(__float_as_uint(p1) & 0xffff0000u)));
+            if constexpr (EB == 2) {
+              pk[i] = __byte_perm(__float_as_uint(p0), __float_as_uint(p1), 0x7632);  // truncate to bf16x2
+              so2 = f32x2_add(so2, f32x2_pack(__uint_as_float(__float_as_uint(p0) & 0xffff0000u),
+                                              __uint_as_float(__float_as_uint(p1) & 0xffff0000u)));
+            } else {
+              // Round to nearest E4M3; four consecutive keys share a column, lowest first.
+              if (i & 1) {
+                pk[i >> 1] = pack_e4m3x4(prev0, prev1, p0, p1);
+              } else {
+                prev0 = p0;
+                prev1 = p1;
+              }
+            }
             sl2 = f32x2_add(sl2, f32x2_pack(p0, p1));
           }
-          tmem_store_16cols(tS + chunk * 16, pk);
+          if constexpr (EB == 2)
+            tmem_store_16cols(tS + chunk * 16, pk);
+          else
+            tmem_store_8cols(tS + chunk * 8, pk);
         }
+        if constexpr (EB == 1) so2 = sl2;  // E4M3: O is normalised by the fp32 sum of p
         float so_lo, so_hi, sl_lo, sl_hi;
         f32x2_unpack(so2, so_lo, so_hi);
         f32x2_unpack(sl2, sl_lo, sl_hi);
@@ -695,7 +736,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
     tc_fence_after_sync();
     if (valid) {
       const bool row_ok = row < p.N;
-      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      const float inv_l = (l_run > 0.f) ? (EB == 2 ? 1.f : p.v_scale) / l_run : 0.f;
       const size_t head_row = (static_cast<size_t>(it.b) * p.Hq + head) * p.N + (row_ok ? row : 0);
       uint4* dst = reinterpret_cast<uint4*>(p.out + head_row * D);
       const uint64_t inv2 = f32x2_pack(inv_l, inv_l);
@@ -725,7 +766,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
           }
         }
       }
-      if (row_ok) p.lse[head_row] = (m_run + __log2f(l_lse) - kP16Bias) * kLn2;
+      if (row_ok) p.lse[head_row] = (m_run + __log2f(l_lse) - kBias) * kLn2;
     }
     tc_fence_before_sync();
     __syncwarp();
@@ -735,9 +776,9 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
   tmem_store_wait();
 }
 
-template <int D>
+template <int D, int EB = 2>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
-  using L = SmemLayout<D>;
+  using L = SmemLayout<D, EB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -779,15 +820,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
   if (warp < 8) {
     reg_alloc_raise<kSoftmaxRegs>();
-    softmax_role<D>(p, sbase, tmem, w, warp, lane);
+    softmax_role<D, EB>(p, sbase, tmem, w, warp, lane);
   } else {
     reg_alloc_lower<kOtherRegs>();
   }
   if (warp == kProducerWarp) {
-    if (lane == 0) producer_role<D>(p, sbase, w);
+    if (lane == 0) producer_role<D, EB>(p, sbase, w);
     __syncwarp();
   } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
-    mma_role<D>(p, sbase, tmem, w, warp - kMmaWarp);
+    mma_role<D, EB>(p, sbase, tmem, w, warp - kMmaWarp);
   }
 
   tc_fence_before_sync();

@@ -1,4 +1,4 @@
-// Thin inline-PTX wrappers for the sm_100a features the attention forward uses:
+// Thin inline-PTX wrappers for the sm_100a features the attention kernels use:
 // mbarriers, TMA tensor loads, tcgen05 (TMEM allocation, MMA, loads/stores,
 // commits and fences), and the global nanosecond timer used by bounded waits.
 // Written from the PTX ISA descriptions of these instructions.
@@ -198,6 +198,40 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
          | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
 }
 
+// Instruction descriptor of kind::f8f6f4: E4M3 A and B (format code 0), fp32
+// accumulator, A K-major; B K-major or MN-major (MN-major is valid for E4M3).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool b_mn_major) {
+  return (1u << 4)                               // D format: f32
+         | (0u << 7)                             // A format: E4M3
+         | (0u << 10)                            // B format: E4M3
+         | ((b_mn_major ? 1u : 0u) << 16)        // B major-ness
+         | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
+}
+
+// kind::f8f6f4 products (K = 32 eight-bit elements = 32 bytes per instruction),
+// warp-uniform with one elected issuing lane like the f16 forms above.
+__device__ __forceinline__ void mma_e4m3_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                  uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_e4m3_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                  uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // TMEM <-> register moves, 32 lanes x 32-bit pattern: thread i of the warp
 // moves row (lane base + i), consecutive registers are consecutive columns.
 // The loads include their wait so the results are valid on return.
@@ -242,6 +276,27 @@ __device__ __forceinline__ void tmem_store_16cols(uint32_t taddr, const uint32_t
       :
       : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
+}
+
+__device__ __forceinline__ void tmem_store_8cols(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+      :
+      : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
+// Four fp32 values to E4M3 (round to nearest, saturating to +-448), a0 in
+// bits 0..7 up to a3 in bits 24..31.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, float a3) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+  return r;
 }
 
 // 32-byte global store (sm_100); ptr must be 32-byte aligned.

@@ -1,5 +1,6 @@
 /*
- * Exact attention forward, backward and paged-KV decoding for NVIDIA B200 (sm_100a): C ABI.
+ * Exact attention forward (bf16 and FP8), backward and paged-KV decoding for NVIDIA B200
+ * (sm_100a): C ABI.
  *
  * Computes, for every batch b, query head h and query row i,
  *
@@ -96,6 +97,30 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* out, float* l
                 float scale, int mask_kind, int64_t window, cudaStream_t stream,
                 const attn_fwd_options* opts);
 
+/*
+ * attn_fwd_fp8: the same forward with E4M3 inputs. q, k, v hold 8-bit E4M3 codes (OCP
+ * format: bias 7, no infinities, largest magnitude 448) in the layouts of attn_fwd, with
+ * one scale per tensor: element value = E4M3(code) * q_scale (k_scale, v_scale). The
+ * result is the exact attention of those values (scale multiplies their q.k), out bf16
+ * and lse fp32 as attn_fwd. The pages name FP8 inputs as a feature of the production
+ * kernel line ("Efficient Attention: Flash Attention, Sliding Window, Sparse",
+ * creativeworksofknowledge.com, section "Flash Attention (exact, memory-efficient)").
+ * Inside, q.k runs on E4M3 tensor-core products and P is rounded to E4M3 (times 2^8)
+ * for the product with V; accumulation is fp32.
+ *
+ *   q, k, v      device pointers to uint8 codes, [B, Hq|Hkv, N, d], contiguous, 16-byte aligned
+ *   q_scale, k_scale, v_scale   finite and > 0
+ *   d            128 only (ATTN_ERR_UNSUPPORTED otherwise)
+ *   everything else as attn_fwd
+ */
+int attn_fwd_fp8(const void* q, const void* k, const void* v, float q_scale, float k_scale, float v_scale,
+                 void* out, float* lse, int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
+                 float scale, int mask_kind, int64_t window, cudaStream_t stream);
+/* attn_fwd_fp8 with options (as attn_fwd_ex); opts may be NULL. */
+int attn_fwd_fp8_ex(const void* q, const void* k, const void* v, float q_scale, float k_scale, float v_scale,
+                    void* out, float* lse, int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
+                    float scale, int mask_kind, int64_t window, cudaStream_t stream,
+                    const attn_fwd_options* opts);
 /* Human-readable name of an attn_status value (static string, never NULL). */
 const char* attn_status_string(int status);
 

@@ -200,3 +200,26 @@ def test_decode_valid_arguments_reach_the_device_check(lib):
     assert call_dec(lib) == 4
     assert call_dec(lib, splits=1) == 4                          # one split: the counter only
     assert call_dec(lib, Nq=40, d=64, page_size=256, mask=2, window=5) == 4
+
+
+# ------------------------------------------------------------------ FP8 forward
+def call_fp8(lib, q=Q, k=K, v=V, o=O, l=L, sq=0.01, sk=0.02, sv=0.03, B=1, Hq=2, Hkv=2, N=256, d=128, scale=0.088,
+             mask=1, window=0):
+    return lib.attn_fwd_fp8(q, k, v, sq, sk, sv, o, l, B, Hq, Hkv, N, d, scale, mask, window, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(v=None), 1), (dict(o=None), 1), (dict(sq=0.0), 1), (dict(sk=-1.0), 1),
+    (dict(sv=float("inf")), 1), (dict(scale=float("nan")), 1), (dict(Hq=3, Hkv=2), 1), (dict(mask=5), 1),
+    (dict(d=64), 2), (dict(d=96), 2), (dict(q=Q + 8), 3), (dict(l=L + 1), 3), (dict(o=K), 1),
+])
+def test_fp8_invalid_arguments_rejected_before_launch(lib, kw, status):
+    assert call_fp8(lib, **kw) == status
+
+
+def test_fp8_valid_arguments_reach_the_device_check(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    assert call_fp8(lib) == 4
+    assert call_fp8(lib, mask=2, window=7) == 4
