@@ -51,7 +51,8 @@ KERNEL_SOURCES = ["exact_io_aware_72_b200/csrc/attn_fwd.cu", "exact_io_aware_72_
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the kernel
 # sources it was taken on; reported only while the sources still match.
 NCU_TRAFFIC = {
-    ("dense", "0d57f4eccd934afc"): 409824768 + 112938752,   # profiles/attn_fwd_dense_ncu.md
+    ("dense", "27db086d122ee63a"): 409273600 + 112365568,       # profiles/attn_fwd_dense_ncu.md
+    ("dense_fp8", "27db086d122ee63a"): 201662464 + 98820864,    # profiles/attn_fwd_fp8_dense_ncu.md
 }
 
 
@@ -81,7 +82,7 @@ DECODE_KERNEL_SOURCES = ["exact_io_aware_72_b200/csrc/attn_decode_kernel.cuh", "
 # DRAM bytes per launch of the decoding kernel from one ncu capture, keyed by
 # workload and the hash of the decoding kernel's device sources.
 DECODE_NCU_TRAFFIC = {
-    ("decode_gqa", "f6e5801ad35ab3ab"): 537009152 + 4729856,   # profiles/attn_decode_gqa_ncu.md
+    ("decode_gqa", "d3ef128b732652ac"): 536993280 + 4117248,   # profiles/attn_decode_gqa_ncu.md
 }
 
 
@@ -371,7 +372,7 @@ def run_ours(args, w):
         achieved = flops / avg_launch_s / 1e12
         peak = float(peaks["bf16_tflops"]) * (FP8_OVER_BF16 if fp8 else 1.0)
         value = world * flops * args.steps / (total_ms / 1e3) / 1e12
-        traffic = None if fp8 else NCU_TRAFFIC.get((w.name, kernel_hash()))
+        traffic = NCU_TRAFFIC.get((w.name + ("_fp8" if fp8 else ""), kernel_hash()))
         line = {
             "metric": FP8_METRIC if fp8 else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
