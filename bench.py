@@ -630,6 +630,60 @@ def run_decode(args, w):
     print(json.dumps(line), flush=True)
 
 
+RING_METRIC = "ring attention TFLOP/s (bf16, causal; all ranks of the ring emulated on one GPU)"
+
+
+def run_ring(args, w):
+    """Ring attention with every rank emulated on one GPU, one after the other:
+    each step runs all ranks' blocks through the forward kernel and their partial
+    results through the merge kernel.  Shows what cutting the sequence into
+    2R halves and merging costs against the single forward of the same workload
+    (no communication happens on one GPU)."""
+    from exact_io_aware_72_b200 import ring
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    R = args.ring_ranks
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, device=device, sharp=w.sharp)
+    shares = ring.emulate_shares(q, k, v, R)
+    del q, k, v
+    flops = workload_flops(w, w.B)
+
+    def step():
+        ring.run_emulated(shares, w.mask, w.scale)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.current_stream(device)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    evs[0].record(stream)
+    for i in range(args.steps):
+        step()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize(device)
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    total_ms = evs[0].elapsed_time(evs[-1])
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    blocks = sum(1 for r in range(R) for s in range(R) for a in ring.half_ids(R, r)
+                 for b in ring.half_ids(R, (r - s) % R) if ring.block_mask(a, b, w.mask) is not None)
+    achieved = flops / (statistics.mean(per) / 1e3) / 1e12
+    line = {
+        "metric": RING_METRIC, "pass": "ring", "value": flops * args.steps / (total_ms / 1e3) / 1e12,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "mask": w.mask,
+                   "ring_ranks": R, "block_rows": w.N // (2 * R), "blocks": blocks,
+                   "l2": "inputs larger than L2 (no flush)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": f"{peak_src} bf16_tflops (burst)"},
+        "gpu_launches": 2 * blocks * args.steps,
+        "launch_ms": {"median": statistics.median(per), "best": min(per)},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -644,9 +698,11 @@ def main():
                     help="B,Hq,Hkv,N,d: run this shape instead of a named workload (profiling sweeps)")
     ap.add_argument("--mask", choices=["full", "causal", "sliding_window"], default=None)
     ap.add_argument("--window", type=int, default=None)
-    ap.add_argument("--pass", dest="which", choices=["fwd", "bwd", "decode"], default="fwd",
-                    help="bwd: the backward pass; decode: a paged-KV decoding step (one GPU each)")
+    ap.add_argument("--pass", dest="which", choices=["fwd", "bwd", "decode", "ring"], default="fwd",
+                    help="bwd: the backward pass; decode: a paged-KV decoding step; ring: ring attention with "
+                         "its ranks emulated on one GPU (one GPU each)")
     ap.add_argument("--splits", type=int, default=0, help="decode: KV splits per sequence (0 = suggested)")
+    ap.add_argument("--ring-ranks", type=int, default=8, help="ring: ranks emulated on the one GPU")
     ap.add_argument("--dtype", choices=["bf16", "fp8"], default="bf16",
                     help="forward inputs: bf16, or E4M3 codes with per-tensor scales")
     args = ap.parse_args()
@@ -669,6 +725,8 @@ def main():
                     window=args.window if mask == "sliding_window" else None, sharp=False)
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.which == "ring":
+        run_ring(args, w)
     elif args.which == "bwd":
         run_backward(args, w)
     else:

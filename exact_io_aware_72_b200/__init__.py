@@ -1,13 +1,15 @@
-"""Exact attention forward (bf16 and FP8 inputs), backward and paged-KV decoding
-for NVIDIA B200 (sm_100a).
+"""Exact attention forward (bf16 and FP8 inputs), backward, paged-KV decoding and
+ring attention across GPUs for NVIDIA B200 (sm_100a).
 
 ``fwd``, ``fwd_fp8``, ``bwd`` and ``decode`` run the hand-written tcgen05/TMA kernels of
 ``libattn_b200.so`` through its C ABI (include/attn.h); there is no CPU or
 library fallback.
 """
 from .attn import (AttnError, MASKS, bwd, bwd_debug_error, debug_error, decode, decode_debug_error,  # noqa: F401
-                   decode_num_splits, decode_workspace_bytes, fwd, fwd_fp8, fwd_host, load_library,
+                   decode_num_splits, decode_workspace_bytes, fwd, fwd_fp8, fwd_host, load_library, merge,
                    num_work_items)
+from . import ring  # noqa: F401
 
 __all__ = ["fwd", "fwd_fp8", "fwd_host", "bwd", "bwd_debug_error", "decode", "decode_debug_error", "decode_num_splits",
-           "decode_workspace_bytes", "debug_error", "load_library", "num_work_items", "AttnError", "MASKS"]
+           "decode_workspace_bytes", "debug_error", "load_library", "merge", "num_work_items", "ring", "AttnError",
+           "MASKS"]

@@ -21,7 +21,7 @@ LIB_NAME = "libattn_b200.so"
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_status_string", "attn_debug_error", "attn_fwd_num_work_items",
            "attn_bwd", "attn_bwd_ex", "attn_bwd_workspace_bytes", "attn_bwd_debug_error",
            "attn_decode", "attn_decode_ex", "attn_decode_workspace_bytes", "attn_decode_num_splits",
-           "attn_decode_debug_error", "attn_fwd_fp8", "attn_fwd_fp8_ex")
+           "attn_decode_debug_error", "attn_fwd_fp8", "attn_fwd_fp8_ex", "attn_merge")
 
 _lib = None
 
@@ -88,6 +88,8 @@ def load_library():
     lib.attn_decode_num_splits.restype = i64
     lib.attn_decode_debug_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.attn_decode_debug_error.restype = ctypes.c_int
+    lib.attn_merge.argtypes = [vp, vp, vp, vp, vp, i64, i64, ctypes.c_int, vp]
+    lib.attn_merge.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -323,6 +325,34 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
     if st != 0:
         raise AttnError(st, "attn_decode")
     return out, lse
+
+
+def merge(acc_out: torch.Tensor, acc_lse: torch.Tensor, part_out: torch.Tensor, part_lse: torch.Tensor,
+          first: bool = False, out: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """Fold a partial attention result (bf16 out, fp32 lse of one block of keys)
+    into an fp32 accumulator in place (``first``: set it instead); when ``out``
+    (bf16) is given the merged rows are also written there."""
+    lib = load_library()
+    if not (acc_out.dtype == torch.float32 and acc_lse.dtype == torch.float32 and part_out.dtype == torch.bfloat16
+            and part_lse.dtype == torch.float32):
+        raise ValueError("merge: acc fp32, part_out bf16, lse fp32")
+    for t, name in ((acc_out, "acc_out"), (acc_lse, "acc_lse"), (part_out, "part_out"), (part_lse, "part_lse")):
+        if not (t.is_cuda and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    d = acc_out.shape[-1]
+    rows = acc_out.numel() // d
+    if part_out.numel() != rows * d or acc_lse.numel() != rows or part_lse.numel() != rows:
+        raise ValueError("merge: shapes disagree")
+    if out is not None and (out.dtype != torch.bfloat16 or not out.is_contiguous() or out.numel() != rows * d):
+        raise ValueError("merge: out must be a contiguous bf16 tensor of the partial's size")
+    if stream is None:
+        stream = torch.cuda.current_stream(acc_out.device)
+    with torch.cuda.device(acc_out.device):
+        st = lib.attn_merge(acc_out.data_ptr(), acc_lse.data_ptr(), part_out.data_ptr(), part_lse.data_ptr(),
+                            out.data_ptr() if out is not None else None, rows, d, 0 if first else 1,
+                            ctypes.c_void_p(stream.cuda_stream))
+    if st != 0:
+        raise AttnError(st, "attn_merge")
 
 
 def decode_debug_error(stream: Optional[torch.cuda.Stream] = None, device=None) -> Tuple[int, int]:

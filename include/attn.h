@@ -1,6 +1,6 @@
 /*
- * Exact attention forward (bf16 and FP8), backward and paged-KV decoding for NVIDIA B200
- * (sm_100a): C ABI.
+ * Exact attention forward (bf16 and FP8), backward, paged-KV decoding and the partial-result
+ * merge of ring attention for NVIDIA B200 (sm_100a): C ABI.
  *
  * Computes, for every batch b, query head h and query row i,
  *
@@ -121,6 +121,27 @@ int attn_fwd_fp8_ex(const void* q, const void* k, const void* v, float q_scale, 
                     void* out, float* lse, int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
                     float scale, int mask_kind, int64_t window, cudaStream_t stream,
                     const attn_fwd_options* opts);
+/*
+ * attn_merge: fold one partial attention result into an accumulator, the combining step of
+ * ring attention ("Attention Mechanism Variants Beyond Self-Attention", tempatgunting.com,
+ * section "Ring Attention for Very Long Sequences": each GPU holds a chunk of the sequence
+ * and key/value blocks rotate around a ring). For each row, with partial (O_p, lse_p) over
+ * one set of keys and accumulated (O_a, lse_a) over a disjoint set,
+ *   lse = ln(e^lse_a + e^lse_p),  O = e^(lse_a - lse) O_a + e^(lse_p - lse) O_p,
+ * the attention over the union (each partial O is normalised by its own softmax sum).
+ *
+ *   acc_out   device, fp32 [rows, d], 16-byte aligned; read (mode 1) and written
+ *   acc_lse   device, fp32 [rows], natural log; read (mode 1) and written
+ *   part_out  device, bf16 [rows, d] (attn_fwd's out for one block of keys), 8-byte aligned
+ *   part_lse  device, fp32 [rows] (attn_fwd's lse for the same block)
+ *   out       device, bf16 [rows, d], 8-byte aligned, or NULL: when given, the merged rows are
+ *             also written here rounded to bf16 (it may be part_out itself)
+ *   rows      1 .. 2^33; d in {64, 128}
+ *   mode      0: the accumulator is set to the partial; 1: the partial is merged into it
+ * Errors as attn_fwd; nothing is allocated and nothing synchronises.
+ */
+int attn_merge(float* acc_out, float* acc_lse, const void* part_out, const float* part_lse, void* out,
+               int64_t rows, int64_t d, int mode, cudaStream_t stream);
 /* Human-readable name of an attn_status value (static string, never NULL). */
 const char* attn_status_string(int status);
 

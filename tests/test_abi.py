@@ -223,3 +223,30 @@ def test_fp8_valid_arguments_reach_the_device_check(lib):
         pytest.skip("GPU present")
     assert call_fp8(lib) == 4
     assert call_fp8(lib, mask=2, window=7) == 4
+
+
+# ------------------------------------------------------------------ partial-result merge
+A1, A2, P1, P2, MO = (0x10000000000 * (i + 20) for i in range(5))
+
+
+def call_merge(lib, acc=A1, accl=A2, part=P1, partl=P2, out=MO, rows=100, d=128, mode=1):
+    return lib.attn_merge(acc, accl, part, partl, out, rows, d, mode, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(acc=None), 1), (dict(accl=None), 1), (dict(part=None), 1), (dict(partl=None), 1),
+    (dict(rows=0), 1), (dict(mode=2), 1), (dict(d=96), 2),
+    (dict(acc=A1 + 8), 3), (dict(part=P1 + 4), 3), (dict(out=MO + 2), 3), (dict(accl=A2 + 2), 3),
+    (dict(accl=A1 + 64), 1), (dict(part=A1), 1), (dict(out=A2), 1), (dict(out=P2), 1),
+])
+def test_merge_invalid_arguments_rejected_before_launch(lib, kw, status):
+    assert call_merge(lib, **kw) == status
+
+
+def test_merge_valid_arguments_reach_the_launch(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    assert call_merge(lib) == 4          # no device: the launch fails
+    assert call_merge(lib, out=None, mode=0) == 4
+    assert call_merge(lib, out=P1) == 4  # out may alias the partial
