@@ -38,8 +38,10 @@
 //   cleared in shared memory before the P V MMA (those slots may hold
 //   anything), and masked scores are replaced by -inf.
 //
-// CTA organisation (192 threads): warps 0-3 softmax (thread = TMEM lane),
-// warp 4 TMA loader, warp 5 tcgen05 issuer.  TMEM: S double buffer at columns
+// CTA organisation (224 threads): warps 0-3 softmax (thread = TMEM lane),
+// warp 4 TMA loader for the work items, Q and K, warp 5 tcgen05 issuer, warp 6
+// TMA loader for V (small pages cost one TMA box each; two issuing warps keep
+// the K and V boxes of a tile going out together).  TMEM: S double buffer at columns
 // [0,128) and [128,256), P double buffer (bf16 pairs) at [256,320) and
 // [320,384), O at [384, 384 + d).  All waits are bounded like the forward's.
 #pragma once
@@ -56,9 +58,10 @@ using namespace attn_sm100;
 
 constexpr int kKeys = 128;           // keys per K/V tile
 constexpr int kLanes = 128;          // query-row lanes of one work item
-constexpr int kDecThreads = 192;
-constexpr int kDecLoaderWarp = 4;
+constexpr int kDecThreads = 224;
+constexpr int kDecLoaderWarp = 4;   // work items, Q and K
 constexpr int kDecMmaWarp = 5;
+constexpr int kDecVLoaderWarp = 6;  // V
 constexpr uint32_t kDecTmemCols = 512;
 constexpr float kDecLn2 = 0.6931471805599453f;
 // A lane's running max moves only when it grows by more than 2^32 (as in the
@@ -244,11 +247,13 @@ __device__ __forceinline__ int dec_take_item(uint32_t sbase, const uint8_t* smem
 }
 
 // ------------------------------------------------------------ roles
-// Loader warp: for every tile of an item, K then V into the next ring slots.
-// Lane i < loads_per_tile copies the tile's rows [i*R, i*R + R) (R =
-// rows_per_load) from the page holding them; lane 0 sets the expected bytes.
-template <int D, int WC>
-__device__ __forceinline__ void dec_loader(const DecParams& p, uint32_t sbase, uint8_t* smem, const DecWaiter& w) {
+// Loader warps: tile t of the CTA's g-th tile overall goes to ring index 2g
+// (K, loader warp 4) and 2g + 1 (V, loader warp 6).  Lane i < loads_per_tile
+// copies the tile's rows [i*R, i*R + R) (R = rows_per_load) from the page
+// holding them; lane 0 sets the expected bytes.  Warp 4 also fetches the work
+// items and loads Q; warp 6 takes the items from it like the other roles.
+template <int D, int WC, bool kV>
+__device__ __forceinline__ uint32_t dec_loader(const DecParams& p, uint32_t sbase, uint8_t* smem, const DecWaiter& w) {
   using L = DecSmem<D>;
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
   const int lane = threadIdx.x & 31;
@@ -261,26 +266,32 @@ __device__ __forceinline__ void dec_loader(const DecParams& p, uint32_t sbase, u
   const int code = kDRoleLoader << 8;
   constexpr int kCopies = 4 / WC;   // replicas of the item's query rows
   constexpr int kRpc = 32 * WC;     // TMEM lanes per replica
-  uint32_t kv_n = 0, q_n = 0, k_item = 0;
+  uint32_t gt = 0, q_n = 0, k_item = 0;  // tiles this CTA has loaded, Q loads, items taken
   bool ok = true;
   // Work items come from the shared counter, one ahead of use so that the
   // atomic's latency overlaps the current item; each index is published to
   // the other roles before the item's loads start.
   int next = 0;
-  if (lane == 0) next = static_cast<int>(atomicAdd(p.sched, 1u));
+  if (!kV && lane == 0) next = static_cast<int>(atomicAdd(p.sched, 1u));
   while (ok) {
-    const uint32_t slot_i = k_item % kItemSlots;
-    if (k_item >= (uint32_t)kItemSlots &&
-        !w.wait_warp(bar(L::kItemEmpty + slot_i), ((k_item / kItemSlots) - 1) & 1, code | (L::kItemEmpty + slot_i)))
-      break;
-    const int idx = __shfl_sync(0xffffffffu, next, 0);
-    if (lane == 0) {
-      *reinterpret_cast<volatile int*>(smem + L::kItemOff + 4 * slot_i) = idx < p.num_items ? idx : -2;
-      mbar_arrive(bar(L::kItemFull + slot_i));
+    int idx;
+    if constexpr (kV) {
+      idx = dec_take_item<D>(sbase, smem, w, k_item, code);
+      if (idx < 0) break;
+    } else {
+      const uint32_t slot_i = k_item % kItemSlots;
+      if (k_item >= (uint32_t)kItemSlots &&
+          !w.wait_warp(bar(L::kItemEmpty + slot_i), ((k_item / kItemSlots) - 1) & 1, code | (L::kItemEmpty + slot_i)))
+        break;
+      idx = __shfl_sync(0xffffffffu, next, 0);
+      if (lane == 0) {
+        *reinterpret_cast<volatile int*>(smem + L::kItemOff + 4 * slot_i) = idx < p.num_items ? idx : -2;
+        mbar_arrive(bar(L::kItemFull + slot_i));
+      }
+      ++k_item;
+      if (idx >= p.num_items) break;
+      if (lane == 0) next = static_cast<int>(atomicAdd(p.sched, 1u));
     }
-    ++k_item;
-    if (idx >= p.num_items) break;
-    if (lane == 0) next = static_cast<int>(atomicAdd(p.sched, 1u));
     const DecItem it = dec_item(p, idx);
     if (it.t1 < it.t0) continue;
     const int* trow = p.block_table + static_cast<size_t>(it.b) * p.max_pages;
@@ -304,9 +315,10 @@ __device__ __forceinline__ void dec_loader(const DecParams& p, uint32_t sbase, u
       return entry;
     };
     auto issue = [&](int t, int kv, int page) -> bool {
-      const uint32_t slot = kv_n % L::kStages;
-      if (kv_n >= (uint32_t)L::kStages &&
-          !w.wait_warp(bar(L::kKVEmpty + slot), ((kv_n / L::kStages) - 1) & 1, code | (L::kKVEmpty + slot)))
+      const uint32_t ring_idx = 2 * gt + kv;
+      const uint32_t slot = ring_idx % L::kStages;
+      if (ring_idx >= (uint32_t)L::kStages &&
+          !w.wait_warp(bar(L::kKVEmpty + slot), ((ring_idx / L::kStages) - 1) & 1, code | (L::kKVEmpty + slot)))
         return false;
       const unsigned boxes = __ballot_sync(0xffffffffu, page >= 0);
       if (lane == 0)
@@ -331,18 +343,18 @@ __device__ __forceinline__ void dec_loader(const DecParams& p, uint32_t sbase, u
                         y, c, z, pol);
         }
       }
-      ++kv_n;
       return true;
     };
     int e0 = box_entry(it.t0), e1 = box_entry(it.t0 + 1);
     for (int t = it.t0; t <= it.t1; ++t) {
       const int e2 = box_entry(t + 2);
       const int pg = checked(t, e0);
-      if (!issue(t, 0, pg) || !issue(t, 1, pg)) {
+      if (!issue(t, kV ? 1 : 0, pg)) {
         ok = false;
         break;
       }
-      if (t == it.t0) {
+      ++gt;
+      if (!kV && t == it.t0) {
         // Q of the item, once the previous item's last S has read the buffer:
         // one box of rows_chunk rows per copy and 64-column chunk.
         if (q_n > 0 && !w.wait_warp(bar(L::kQEmpty), (q_n - 1) & 1, code | L::kQEmpty)) {
@@ -365,17 +377,30 @@ __device__ __forceinline__ void dec_loader(const DecParams& p, uint32_t sbase, u
       e1 = e2;
     }
   }
-  // Drain: every copy this warp started must land before the CTA exits.
-  if (lane == 0) {
-    for (uint32_t s = 0; s < (uint32_t)L::kStages; ++s) {
-      if (kv_n > s) {
-        const uint32_t last = s + ((kv_n - 1 - s) / L::kStages) * L::kStages;
-        w.drain(bar(L::kKVFull + s), (last / L::kStages) & 1, code | (L::kKVFull + s));
-      }
-    }
-    if (q_n > 0) w.drain(bar(L::kQFull), (q_n - 1) & 1, code | L::kQFull);
-  }
+  // Drain this warp's Q copies; the K/V ring is drained after both loaders
+  // are done (dec_drain_ring), since the two warps take turns on every slot.
+  if (lane == 0 && q_n > 0) w.drain(bar(L::kQFull), (q_n - 1) & 1, code | L::kQFull);
   __syncwarp();
+  return gt;
+}
+
+// Every K/V copy must land before the CTA exits.  A slot is loaded again only
+// after its previous load landed and was consumed, so at most its last load
+// can still be in flight: wait for that one (ring index 2g for K, 2g + 1 for V).
+template <int D>
+__device__ __forceinline__ void dec_drain_ring(uint32_t sbase, const DecWaiter& w, uint32_t gt_k, uint32_t gt_v) {
+  using L = DecSmem<D>;
+  for (uint32_t s = 0; s < (uint32_t)L::kStages; ++s) {
+    int64_t last = -1;
+    for (uint32_t back = 0; back < (uint32_t)L::kStages; ++back) {
+      if (back < gt_k && (2 * (gt_k - 1 - back)) % L::kStages == s) last = max(last, int64_t(2 * (gt_k - 1 - back)));
+      if (back < gt_v && (2 * (gt_v - 1 - back) + 1) % L::kStages == s)
+        last = max(last, int64_t(2 * (gt_v - 1 - back) + 1));
+    }
+    if (last >= 0)
+      w.drain(sbase + L::kBarOff + 8u * (L::kKVFull + s), (uint32_t(last) / L::kStages) & 1,
+              (kDRoleLoader << 8) | (L::kKVFull + s));
+  }
 }
 
 // MMA warp: per item S_0, then for each tile j: S_{j+1} (look-ahead into the
@@ -740,6 +765,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
   const int warp = threadIdx.x >> 5;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  volatile uint32_t* loaded = reinterpret_cast<volatile uint32_t*>(smem + L::kMiscOff + 8);  // tiles per loader
 
   // Query-buffer rows that no Q box covers must read as zero.
   for (uint32_t i = threadIdx.x; i < L::kTileBytes / 16; i += kDecThreads)
@@ -764,7 +790,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
     mbar_init(bar(L::kFin), 1);
     for (int i = 0; i < kItemSlots; ++i) {
       mbar_init(bar(L::kItemFull + i), 1);
-      mbar_init(bar(L::kItemEmpty + i), 5);  // the MMA warp and the four softmax warps
+      mbar_init(bar(L::kItemEmpty + i), 6);  // the MMA warp, the four softmax warps and the V loader
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -782,13 +808,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
   if (warp < 4) {
     dec_softmax<D, WC>(p, sbase, smem, tmem, w);
   } else if (warp == kDecLoaderWarp) {
-    dec_loader<D, WC>(p, sbase, smem, w);
+    const uint32_t gt = dec_loader<D, WC, false>(p, sbase, smem, w);
+    if ((threadIdx.x & 31) == 0) loaded[0] = gt;
+  } else if (warp == kDecVLoaderWarp) {
+    const uint32_t gt = dec_loader<D, WC, true>(p, sbase, smem, w);
+    if ((threadIdx.x & 31) == 0) loaded[1] = gt;
   } else {
     dec_mma<D>(p, sbase, smem, tmem, w);
   }
 
   tc_fence_before_sync();
   __syncthreads();
+  if (threadIdx.x == kDecLoaderWarp * 32) dec_drain_ring<D>(sbase, w, loaded[0], loaded[1]);
   if (warp == kDecMmaWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, kDecTmemCols);
