@@ -82,7 +82,7 @@ DECODE_KERNEL_SOURCES = ["exact_io_aware_72_b200/csrc/attn_decode_kernel.cuh", "
 # DRAM bytes per launch of the decoding kernel from one ncu capture, keyed by
 # workload and the hash of the decoding kernel's device sources.
 DECODE_NCU_TRAFFIC = {
-    ("decode_gqa", "d3ef128b732652ac"): 536993280 + 4117248,   # profiles/attn_decode_gqa_ncu.md
+    ("decode_gqa", "32d09ba4e712aaae"): 536997632 + 3341312,   # profiles/attn_decode_gqa_ncu.md
 }
 
 
