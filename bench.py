@@ -7,13 +7,16 @@ visible (query, key) pair.  Inputs (384 MiB of q, k, v) are larger than the
 126 MB L2, so no flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload dense|gqa|swa|long|tiny] [--no-cpu-baseline] [--pass fwd|bwd|decode]
+                  [--workload dense|gqa|swa|long|tiny|decode_*] [--no-cpu-baseline]
+                  [--pass fwd|bwd|decode|ring] [--dtype bf16|fp8]
 
 ``--pass bwd`` times the backward pass instead (one GPU; 10*d FLOPs per visible
 pair, the five products of the gradient).  ``--pass decode`` times one decoding
 step against a paged KV cache (``--workload decode_gqa|decode_mha|decode_swa|
 decode_spec``; one GPU; GB/s of algorithmic bytes against the measured HBM
-bandwidth).
+bandwidth).  ``--dtype fp8`` runs the forward on E4M3 inputs (peak: the measured bf16
+figure x 2).  ``--pass ring`` runs ring attention with all its ranks emulated on one GPU
+(``--ring-ranks R``).
 
 With --gpus N > 1 the script runs under torchrun, one rank per GPU; every rank
 runs its own shard of the global batch (weak scaling, no data-path collective)

@@ -21,8 +21,7 @@ What it computes, restated from the pages:
   forward (``oracle.attention_fp64``): causal j <= i, sliding window
   i - w < j <= i, or every cached key.
 
-Readings where the pages leave the step open (each also listed in the design
-notes):
+Readings where the pages leave the step open:
 
 * Layouts: q ``[B, Hq, Nq, d]``; each cache ``[num_pages, Hkv, page_size, d]``
   (one page holds ``page_size`` consecutive positions of every KV head);

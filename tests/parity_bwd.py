@@ -1,7 +1,6 @@
 """Element-wise parity of the CUDA backward with the fp64 backward oracle.
 
-Bound (derived from the arithmetic of the CUDA path, stated again in the
-design notes): the kernels recompute P = exp(S - lse) in fp32, round P and
+Bound (derived from the arithmetic of the CUDA path): the kernels recompute P = exp(S - lse) in fp32, round P and
 dS = P (dP - D) to bf16 (relative error <= 2^-9 each, round to nearest) before
 the P^T dO, dS K and dS^T Q products, take D from the forward's bf16 output O
 (|D - D_exact| <= 2^-9 sum_c |dO_c O_c|), accumulate in fp32 and round each
