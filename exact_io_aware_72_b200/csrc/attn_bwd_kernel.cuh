@@ -427,6 +427,7 @@ __device__ __forceinline__ void dq_elem(const BwdParams& p, uint32_t sbase, uint
     const size_t bhrow = (static_cast<size_t>(it.b) * p.Hq + it.hq) * p.N + (row_ok ? row : 0);
     const float lse2 = row_ok ? p.lse[bhrow] * kLog2e : 0.f;
     const float dlt = row_ok ? p.delta[bhrow] : 0.f;
+    const uint64_t c2x2 = f32x2_pack(c2, c2), nlse2x2 = f32x2_pack(-lse2, -lse2), ndlt2 = f32x2_pack(-dlt, -dlt);
     bool ok = true;
     for (int j = it.lo; j <= it.hi && ok; ++j, ++s_cnt) {
       const bool partial = block_is_partial(p, it.m, j);
@@ -457,13 +458,16 @@ __device__ __forceinline__ void dq_elem(const BwdParams& p, uint32_t sbase, uint
           }
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            float ds[2];
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-              const float pr = bexp2(__uint_as_float(sv[e + x]) * c2 - lse2);
-              ds[x] = pr * (__uint_as_float(pv[e + x]) - dlt);
-            }
-            packed[chunk][e >> 1] = bf16x2_rn(ds[0], ds[1]);
+            // Column pairs on packed fp32 operations: x = s c - lse, p = 2^x,
+            // dS = p (dP - D).
+            float x0, x1, d0, d1;
+            f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2x2, nlse2x2),
+                         x0, x1);
+            const uint64_t pr2 = f32x2_pack(bexp2(x0), bexp2(x1));
+            f32x2_unpack(f32x2_mul(pr2, f32x2_add(f32x2_pack(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1])),
+                                                  ndlt2)),
+                         d0, d1);
+            packed[chunk][e >> 1] = bf16x2_rn(d0, d1);
           }
         }
         // dS (bf16, 32 columns) over the first half of this half's S columns.
@@ -646,10 +650,12 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
   const int r = warp * 32 + lane;  // key row of the tile = TMEM lane
   const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t t_dv = tmem + lane_bits + L::kColAcc0, t_dk = tmem + lane_bits + L::kColAcc1;
-  // This warp's copy of the step's log2-scaled LSE and D of the 128 query rows.
+  // This warp's copy of the step's log2-scaled LSE and D of the 128 query
+  // rows, both negated (they are subtracted).
   float* s_lse = reinterpret_cast<float*>(__cvta_shared_to_generic(sbase + L::kVecOff)) + warp * 2 * kTile;
   float* s_dlt = s_lse + kTile;
   const float c2 = p.scale_log2;
+  const uint64_t c2x2 = f32x2_pack(c2, c2);
   const int code = (kBKernelDkdv << 12) | (kBRoleElem << 8);
   uint32_t s_cnt = 0;
   int items = 0;
@@ -666,8 +672,8 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const int c = lane + 32 * t, q = m * kTile + c;
-          s_lse[c] = (q < p.N) ? p.lse[bhq + q] * kLog2e : 0.f;
-          s_dlt[c] = (q < p.N) ? p.delta[bhq + q] : 0.f;
+          s_lse[c] = (q < p.N) ? -p.lse[bhq + q] * kLog2e : 0.f;
+          s_dlt[c] = (q < p.N) ? -p.delta[bhq + q] : 0.f;
         }
         __syncwarp();
       }
@@ -700,15 +706,23 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
           }
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            float pr[2], ds[2];
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-              const int c = h * kHalf + chunk * 32 + e + x;  // query column within the tile
-              pr[x] = bexp2(__uint_as_float(sv[e + x]) * c2 - s_lse[c]);
-              ds[x] = pr[x] * (__uint_as_float(pv[e + x]) - s_dlt[c]);
-            }
-            pk[chunk][e >> 1] = bf16x2_rn(pr[0], pr[1]);
-            dk[chunk][e >> 1] = bf16x2_rn(ds[0], ds[1]);
+            // Column pairs: x = s c - lse, p = 2^x, dS = p (dP - D), with the
+            // pair's (-lse, -D) read as 8-byte loads and packed fp32 arithmetic.
+            const int c = h * kHalf + chunk * 32 + e;  // query column within the tile (even)
+            const float2 nl = *reinterpret_cast<const float2*>(s_lse + c);
+            const float2 nd = *reinterpret_cast<const float2*>(s_dlt + c);
+            float x0, x1, p0, p1, d0, d1;
+            f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2x2,
+                                   f32x2_pack(nl.x, nl.y)),
+                         x0, x1);
+            p0 = bexp2(x0);
+            p1 = bexp2(x1);
+            f32x2_unpack(f32x2_mul(f32x2_pack(p0, p1), f32x2_add(f32x2_pack(__uint_as_float(pv[e]),
+                                                                            __uint_as_float(pv[e + 1])),
+                                                                f32x2_pack(nd.x, nd.y))),
+                         d0, d1);
+            pk[chunk][e >> 1] = bf16x2_rn(p0, p1);
+            dk[chunk][e >> 1] = bf16x2_rn(d0, d1);
           }
         }
         // P^T and dS^T (bf16, 32 columns each) over the first halves of this
