@@ -161,3 +161,11 @@ def test_shared_workspace_counter_returns_to_zero(cuda_ok):
             if ref is None:
                 ref = oracle_for({k: v.cpu() for k, v in inp.items()}, "causal")
             compare(to_np(out), to_np(lse), ref[0], ref[1], f"splits {splits} grid {grid}")
+
+
+@pytest.mark.parametrize("Nq,window", [(3, None), (5, 100), (2, 1)])
+def test_head_dim_64_multi_token_and_window(cuda_ok, Nq, window):
+    lens = [Nq, 130, 999, 2500]
+    mask = "causal" if window is None else "sliding_window"
+    check_decode_case(len(lens), 8, 2, Nq, 64, lens, 32, mask, window=window, seed=Nq + 7, num_splits=2,
+                      rolling=window is not None)

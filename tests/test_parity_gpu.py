@@ -125,3 +125,19 @@ def test_out_16_byte_aligned_matches_32_byte_aligned_bitwise(cuda_ok):
     fwd(q, k, v, mask="causal", out=out, lse=lse)
     torch.cuda.synchronize()
     assert torch.equal(out, o_ref) and torch.equal(lse, l_ref)
+
+
+@pytest.mark.parametrize("shape", [(64, 2, 1, 64, 128), (33, 3, 3, 129, 64), (1, 96, 8, 200, 128)])
+def test_many_small_heads_and_sequences(cuda_ok, shape):
+    # far more work items than SMs, each tiny: the static schedule's tail split
+    B, Hq, Hkv, N, d = shape
+    check_case(B, Hq, Hkv, N, d, "causal", seed=B + Hq + N)
+
+
+def test_grid_sizes_give_identical_bits(cuda_ok):
+    from exact_io_aware_72_b200 import fwd
+    q, k, v = (t.cuda() for t in make_qkv(2, 8, 2, 1000, 128, 21))
+    ref = fwd(q, k, v)
+    for grid in (1, 5, 37, 148):
+        got = fwd(q, k, v, grid_ctas=grid)
+        assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1])
