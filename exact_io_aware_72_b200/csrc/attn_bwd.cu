@@ -109,8 +109,7 @@ bool sizes_ok(int64_t B, int64_t Hq, int64_t Hkv, int64_t N) {
 
 template <int D, int KIND>
 cudaError_t launch_bwd(const BwdParams& p, int grid, cudaStream_t stream) {
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kBwdThreads);
   cfg.dynamicSmemBytes = BwdSmem<D>::kAlloc;

@@ -113,8 +113,7 @@ size_t workspace_bytes(int64_t rows, int64_t d, int64_t splits) {
 
 template <int D, int WC>
 cudaError_t launch_decode(const DecParams& p, int grid, cudaStream_t stream) {
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kDecThreads);
   cfg.dynamicSmemBytes = DecSmem<D>::kAlloc;

@@ -204,8 +204,7 @@ int fwd_launch(const void* q, const void* k, const void* v, void* out, float* ls
   if (opts && opts->grid_ctas > 0) grid = opts->grid_ctas;
   if (grid > plan.super_items) grid = static_cast<int>(plan.super_items);
 
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
   cfg.stream = stream;
