@@ -227,9 +227,19 @@ def cpu_baseline(w, q, k, v, target_s=15.0):
                            count=min(w.N, int(len(rows) * target_s / max(dt * n_heads, 1e-3) / 2)))
     heads = [(i // w.Hq, i % w.Hq) for i in range(n_heads)]
     dt, flops, threads = oracle_sample(w, q, k, v, rows, heads, w.scale)
+    # The same oracle on one thread, on a smaller sample (one head, up to 64 rows).
+    from threadpoolctl import threadpool_limits
+    rows1 = rows[:: max(1, len(rows) // 64)][:64]
+    with threadpool_limits(limits=1):
+        dt1, flops1, _ = oracle_sample(w, q, k, v, rows1, heads[:1], w.scale)
+    pairs = flops // (4 * w.d)
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "rows_per_s": len(rows) * n_heads / dt, "pairs_per_s": pairs / dt,
+            "one_thread": {"value": flops1 / dt1 / 1e12, "unit": "TFLOP/s", "rows_per_s": len(rows1) / dt1,
+                           "pairs_per_s": flops1 // (4 * w.d) / dt1},
             "sample": f"{len(rows)} seeded query rows x {n_heads} heads of the {w.name} workload "
-                      f"(fp64 NumPy, scores materialised), {dt:.1f} s",
+                      f"(fp64 NumPy, scores materialised), {dt:.1f} s; one thread: {len(rows1)} rows of "
+                      f"one head, {dt1:.2f} s",
             "seconds": dt}
 
 
