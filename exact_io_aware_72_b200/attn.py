@@ -21,7 +21,8 @@ LIB_NAME = "libattn_b200.so"
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_status_string", "attn_debug_error", "attn_fwd_num_work_items",
            "attn_bwd", "attn_bwd_ex", "attn_bwd_workspace_bytes", "attn_bwd_debug_error",
            "attn_decode", "attn_decode_ex", "attn_decode_workspace_bytes", "attn_decode_num_splits",
-           "attn_decode_debug_error", "attn_fwd_fp8", "attn_fwd_fp8_ex", "attn_merge")
+           "attn_decode_debug_error", "attn_fwd_fp8", "attn_fwd_fp8_ex", "attn_merge", "attn_fwd_host",
+           "attn_fwd_fp8_host")
 
 _lib = None
 
@@ -88,6 +89,11 @@ def load_library():
     lib.attn_decode_num_splits.restype = i64
     lib.attn_decode_debug_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.attn_decode_debug_error.restype = ctypes.c_int
+    host_tail = [vp] * 7 + [i64] * 5 + [f32, ctypes.c_int, i64, i64, vp]
+    lib.attn_fwd_host.argtypes = [vp, vp, vp] + host_tail
+    lib.attn_fwd_host.restype = ctypes.c_int
+    lib.attn_fwd_fp8_host.argtypes = [vp, vp, vp, f32, f32, f32] + host_tail
+    lib.attn_fwd_fp8_host.restype = ctypes.c_int
     lib.attn_merge.argtypes = [vp, vp, vp, vp, vp, i64, i64, ctypes.c_int, vp]
     lib.attn_merge.restype = ctypes.c_int
     _lib = lib
@@ -377,20 +383,82 @@ def debug_error(stream: Optional[torch.cuda.Stream] = None, device=None) -> Tupl
     return st, code.value
 
 
-def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, device="cuda", **kw):
-    """End-to-end call on HOST tensors (ideally pinned): copies q, k, v to the
-    device, runs the forward, and copies out and lse back to host memory."""
-    dq = q.to(device, non_blocking=True)
-    dk = k.to(device, non_blocking=True)
-    dv = v.to(device, non_blocking=True)
-    out, lse = fwd(dq, dk, dv, **kw)
+def _host_tensor(t, name: str, dtype) -> torch.Tensor:
+    if isinstance(t, torch.Tensor) and t.dtype == torch.float8_e4m3fn and dtype == torch.uint8:
+        t = t.view(torch.uint8)
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or t.dim() != 4 or t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous host {dtype} tensor with 4 dims")
+    return t
+
+
+def _fwd_host(fp8: bool, q, k, v, q_scale, k_scale, v_scale, scale, mask, window, chunks, device, out, lse,
+              staging, stream):
+    lib = load_library()
+    dt = torch.uint8 if fp8 else torch.bfloat16
+    q, k, v = _host_tensor(q, "q", dt), _host_tensor(k, "k", dt), _host_tensor(v, "v", dt)
+    B, Hq, N, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if (Bk, Nk, dk) != (B, N, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("q, k, v shapes disagree")
+    if mask not in MASKS:
+        raise ValueError(f"mask must be one of {sorted(MASKS)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
     pin = q.is_pinned()
-    ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=pin)
-    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=pin)
-    ho.copy_(out, non_blocking=True)
-    hl.copy_(lse, non_blocking=True)
-    torch.cuda.current_stream(dq.device).synchronize()
-    return ho, hl
+    if out is None:
+        out = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, pin_memory=pin)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, pin_memory=pin)
+    if out.is_cuda or lse.is_cuda or out.dtype != torch.bfloat16 or lse.dtype != torch.float32 or \
+            tuple(out.shape) != (B, Hq, N, d) or tuple(lse.shape) != (B, Hq, N) or \
+            not out.is_contiguous() or not lse.is_contiguous():
+        raise ValueError("out and lse must be contiguous host tensors: bf16 [B,Hq,N,d] and fp32 [B,Hq,N]")
+    device = torch.device(device)
+    if staging is None:
+        staging = (torch.empty(q.shape, dtype=dt, device=device), torch.empty(k.shape, dtype=dt, device=device),
+                   torch.empty(k.shape, dtype=dt, device=device),
+                   torch.empty(out.shape, dtype=torch.bfloat16, device=device),
+                   torch.empty(lse.shape, dtype=torch.float32, device=device))
+    sq, sk, sv, so, sl = staging
+    for t, ref, name in ((sq, q, "q"), (sk, k, "k"), (sv, v, "v"), (so, out, "out"), (sl, lse, "lse")):
+        if not t.is_cuda or t.dtype != ref.dtype or tuple(t.shape) != tuple(ref.shape) or not t.is_contiguous():
+            raise ValueError(f"staging buffer for {name} must be a contiguous CUDA tensor like it")
+    if stream is None:
+        stream = torch.cuda.current_stream(sq.device)
+    common = (out.data_ptr(), lse.data_ptr(), sq.data_ptr(), sk.data_ptr(), sv.data_ptr(), so.data_ptr(),
+              sl.data_ptr(), B, Hq, Hkv, N, d, float(scale), MASKS[mask],
+              int(window) if window is not None else 0, int(chunks), ctypes.c_void_p(stream.cuda_stream))
+    with torch.cuda.device(sq.device):
+        if fp8:
+            st = lib.attn_fwd_fp8_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), float(q_scale), float(k_scale),
+                                       float(v_scale), *common)
+        else:
+            st = lib.attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), *common)
+    if st != 0:
+        raise AttnError(st, "attn_fwd_fp8_host" if fp8 else "attn_fwd_host")
+    stream.synchronize()
+    return out, lse
+
+
+def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
+             mask: str = "causal", window: Optional[int] = None, chunks: int = 0, device="cuda",
+             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, staging=None,
+             stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The forward on HOST tensors (pinned for overlapped copies), end to end:
+    q, k, v go up and out, lse come back in ``chunks`` pieces whose copies
+    overlap the kernels (``attn_fwd_host``).  ``staging`` optionally gives the
+    device buffers (dq, dk, dv, dout, dlse); returns host (out, lse), complete."""
+    return _fwd_host(False, q, k, v, 1.0, 1.0, 1.0, scale, mask, window, chunks, device, out, lse, staging, stream)
+
+
+def fwd_fp8_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_scale: float, k_scale: float,
+                 v_scale: float, scale: Optional[float] = None, mask: str = "causal", window: Optional[int] = None,
+                 chunks: int = 0, device="cuda", out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None, staging=None, stream: Optional[torch.cuda.Stream] = None
+                 ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """``fwd_host`` for the E4M3 codes of ``fwd_fp8`` (``attn_fwd_fp8_host``)."""
+    return _fwd_host(True, q, k, v, q_scale, k_scale, v_scale, scale, mask, window, chunks, device, out, lse,
+                     staging, stream)
 
 
 def num_work_items(B, Hq, Hkv, N, d, mask="causal", window=None) -> int:

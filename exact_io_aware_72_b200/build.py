@@ -9,7 +9,8 @@ PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 LIB_PATH = os.path.join(PKG_DIR, "libattn_b200.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("attn_fwd.cu", "attn_bwd.cu", "attn_decode.cu", "attn_merge.cu")]
+SOURCES = [os.path.join(CSRC, f) for f in ("attn_fwd.cu", "attn_bwd.cu", "attn_decode.cu", "attn_merge.cu",
+                                                "attn_fwd_host.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in ("attn_fwd_kernel.cuh", "attn_bwd_kernel.cuh", "attn_decode_kernel.cuh", "sm100_ptx.cuh")] + [
     os.path.join(ROOT, "include", "attn.h")]
 

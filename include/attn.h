@@ -121,6 +121,44 @@ int attn_fwd_fp8_ex(const void* q, const void* k, const void* v, float q_scale, 
                     void* out, float* lse, int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
                     float scale, int mask_kind, int64_t window, cudaStream_t stream,
                     const attn_fwd_options* opts);
+
+/*
+ * attn_fwd_host: attn_fwd on HOST buffers, with the copies overlapped with the work.
+ * The (batch, key/value head) units are independent and a contiguous range of units is a
+ * contiguous range of every tensor, so the job is cut into `chunks` ranges. Each range is
+ * uploaded on a copy stream. Its forward runs on `stream` once it has arrived, and its out
+ * and lse go back on a second copy stream once computed. Different chunks' uploads, kernels
+ * and downloads therefore run at the same time.
+ *
+ *   hq, hk, hv    host pointers, layouts and types of attn_fwd's q, k, v (page-locked
+ *                 memory lets the copies overlap; pageable memory works, more slowly)
+ *   hout, hlse    host pointers, layouts of attn_fwd's out and lse; must not overlap the
+ *                 host inputs or each other
+ *   dq, dk, dv, dout, dlse   device staging buffers with attn_fwd's sizes, alignment and
+ *                 overlap rules (owned by the caller; their contents are overwritten)
+ *   B ... window  as attn_fwd
+ *   chunks        number of ranges, >= 0; 0 = 8; more than B * Hkv means B * Hkv
+ *   stream        CUDA stream of the current device
+ *
+ * Everything is enqueued and the call returns. hout and hlse are complete when `stream`
+ * reaches the point after the call: `stream` waits for the last download. The call does
+ * not block the host unless the host memory is pageable, in which case the runtime may
+ * copy synchronously. The library keeps two copy streams per device, created on first
+ * use, and allocates no memory. Errors: arguments are checked before anything is
+ * enqueued, as in attn_fwd. If a copy or launch fails part way, ATTN_ERR_CUDA is
+ * returned; `stream` is still ordered after whatever had been enqueued.
+ */
+int attn_fwd_host(const void* hq, const void* hk, const void* hv, void* hout, float* hlse,
+                  void* dq, void* dk, void* dv, void* dout, float* dlse,
+                  int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
+                  float scale, int mask_kind, int64_t window, int64_t chunks, cudaStream_t stream);
+/* attn_fwd_host for the E4M3 inputs of attn_fwd_fp8 (same scales, same restrictions). */
+int attn_fwd_fp8_host(const void* hq, const void* hk, const void* hv,
+                      float q_scale, float k_scale, float v_scale, void* hout, float* hlse,
+                      void* dq, void* dk, void* dv, void* dout, float* dlse,
+                      int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
+                      float scale, int mask_kind, int64_t window, int64_t chunks, cudaStream_t stream);
+
 /*
  * attn_merge: fold one partial attention result into an accumulator, the combining step of
  * ring attention ("Attention Mechanism Variants Beyond Self-Attention", tempatgunting.com,

@@ -250,3 +250,38 @@ def test_merge_valid_arguments_reach_the_launch(lib):
     assert call_merge(lib) == 4          # no device: the launch fails
     assert call_merge(lib, out=None, mode=0) == 4
     assert call_merge(lib, out=P1) == 4  # out may alias the partial
+
+
+# ------------------------------------------------------------------ host-buffer forward
+HQ, HK, HV, HO, HL = (0x10000000000 * (i + 40) for i in range(5))
+
+
+def call_host(lib, hq=HQ, hk=HK, hv=HV, ho=HO, hl=HL, q=Q, k=K, v=V, o=O, l=L, B=2, Hq=4, Hkv=2, N=256, d=64,
+              scale=0.125, mask=1, window=0, chunks=0, fp8=False, sq=0.01, sk=0.02, sv=0.03):
+    if fp8:
+        return lib.attn_fwd_fp8_host(hq, hk, hv, sq, sk, sv, ho, hl, q, k, v, o, l, B, Hq, Hkv, N, d, scale, mask,
+                                     window, chunks, None)
+    return lib.attn_fwd_host(hq, hk, hv, ho, hl, q, k, v, o, l, B, Hq, Hkv, N, d, scale, mask, window, chunks, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(hq=None), 1), (dict(hv=None), 1), (dict(ho=None), 1), (dict(hl=None), 1), (dict(q=None), 1),
+    (dict(l=None), 1), (dict(B=0), 1), (dict(Hq=3), 1), (dict(mask=4), 1), (dict(mask=2, window=0), 1),
+    (dict(scale=0.0), 1), (dict(chunks=-1), 1), (dict(d=96), 2),
+    (dict(q=Q + 8), 3), (dict(o=O + 4), 3), (dict(l=L + 2), 3),
+    (dict(o=K), 1), (dict(l=O + 64), 1),                        # device outputs overlap
+    (dict(ho=HQ + 1024), 1), (dict(hl=HO + 4096), 1), (dict(hl=HV), 1),   # host outputs overlap
+    (dict(fp8=True, d=64), 2), (dict(fp8=True, d=128, sq=0.0), 1), (dict(fp8=True, d=128, sv=float("nan")), 1),
+])
+def test_host_forward_invalid_arguments_rejected_before_enqueueing(lib, kw, status):
+    assert call_host(lib, **kw) == status
+
+
+def test_host_forward_valid_arguments_reach_the_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    assert call_host(lib) == 4                       # no device: the copy streams cannot be made
+    assert call_host(lib, hq=HQ + 3, ho=HO + 2) == 4  # host buffers need no alignment
+    assert call_host(lib, chunks=100) == 4
+    assert call_host(lib, fp8=True, d=128) == 4
