@@ -1,6 +1,6 @@
 /*
- * Exact attention forward (bf16 and FP8), backward, paged-KV decoding and the partial-result
- * merge of ring attention for NVIDIA B200 (sm_100a): C ABI.
+ * Exact attention forward (bf16 and FP8, on device or host buffers), backward, paged-KV
+ * decoding and the partial-result merge of ring attention for NVIDIA B200 (sm_100a): C ABI.
  *
  * Computes, for every batch b, query head h and query row i,
  *
