@@ -280,6 +280,8 @@ def run_reference(args, w):
         total_s += dt
         total_f += fl
     value = total_f / total_s / 1e12
+    rows_per_s = len(rows) * len(heads) * args.steps / total_s
+    pairs_per_s = total_f / (4 * w.d) / total_s
     sample = f"{len(rows)} seeded query rows x {len(heads)} heads of the {w.name} workload per step (fp64 NumPy)"
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000 * total_s / args.steps, "higher_is_better": True,
@@ -289,7 +291,7 @@ def run_reference(args, w):
                        "mask": w.mask, "window": w.window, "global_batch": w.B, "seq_len": w.N,
                        "parallelism": "cpu"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                             "sample": sample},
+                             "rows_per_s": rows_per_s, "pairs_per_s": pairs_per_s, "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
