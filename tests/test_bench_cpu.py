@@ -78,3 +78,27 @@ def test_workload_flops_are_four_d_per_visible_pair():
     # the long workload: N = 131072, d = 128, 32 heads, causal
     w = WORKLOADS["long"]
     assert bench.workload_flops(w, 1) == 4 * 32 * 128 * (131072 * 131073 // 2)
+
+
+def _brute_decode_keys(L, Nq, mask, window):
+    """Positions j < L that at least one of the step's queries (positions L-Nq .. L-1) sees."""
+    seen = set()
+    for i in range(L - Nq, L):
+        for j in range(L):
+            if mask == "full" or (mask == "causal" and j <= i) or \
+                    (mask == "sliding_window" and i - window < j <= i):
+                seen.add(j)
+    return len(seen)
+
+
+@pytest.mark.parametrize("mask,window,Nq", [("causal", None, 1), ("causal", None, 4), ("full", None, 2),
+                                            ("sliding_window", 1, 1), ("sliding_window", 7, 3),
+                                            ("sliding_window", 50, 4), ("sliding_window", 500, 2)])
+def test_decode_bytes_count_the_visible_cached_positions(mask, window, Nq):
+    from dataclasses import replace
+    from harness.inputs import DECODE_WORKLOADS
+    lens = [Nq, Nq + 1, 37, 64, 129, 300]
+    w = replace(DECODE_WORKLOADS["decode_gqa"], B=len(lens), Nq=Nq, mask=mask, window=window)
+    keys = sum(_brute_decode_keys(L, Nq, mask, window) for L in lens)
+    expect = 2 * 2 * w.d * w.Hkv * keys + w.B * w.Hq * Nq * (2 * 2 * w.d + 4)
+    assert bench.decode_bytes(w, lens) == expect
