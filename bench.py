@@ -661,21 +661,38 @@ def run_ring(args, w):
     del q, k, v
     flops = workload_flops(w, w.B)
 
-    def step():
+    def eager_step():
         ring.run_emulated(shares, w.mask, w.scale)
 
     for _ in range(args.warmup):
-        step()
+        eager_step()
     torch.cuda.synchronize(device)
     stream = torch.cuda.current_stream(device)
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    evs[0].record(stream)
-    for i in range(args.steps):
-        step()
-        evs[i + 1].record(stream)
-    torch.cuda.synchronize(device)
-    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
-    total_ms = evs[0].elapsed_time(evs[-1])
+
+    def timed(step):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        evs[0].record(stream)
+        for i in range(args.steps):
+            step()
+            evs[i + 1].record(stream)
+        torch.cuda.synchronize(device)
+        return [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)], evs[0].elapsed_time(evs[-1])
+
+    eager_per, eager_ms = timed(eager_step)
+    # The step's launches (one forward and one merge per block) captured once in a
+    # CUDA graph and replayed: small blocks are otherwise bound by the host's
+    # launch path, not by the GPU.
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            ring.run_emulated(shares, w.mask, w.scale)
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize(device)
+        per, total_ms = timed(graph.replay)
+    else:
+        per, total_ms = eager_per, eager_ms
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
     blocks = sum(1 for r in range(R) for s in range(R) for a in ring.half_ids(R, r)
@@ -688,7 +705,10 @@ def run_ring(args, w):
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "mask": w.mask,
                    "ring_ranks": R, "block_rows": w.N // (2 * R), "blocks": blocks,
+                   "launch": "cuda_graph" if graph is not None else "eager",
                    "l2": "inputs larger than L2 (no flush)"},
+        "eager": {"value": flops * args.steps / (eager_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                  "ms_per_step": eager_ms / args.steps},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "traffic": None, "peak_source": f"{peak_src} bf16_tflops (burst)"},
         "gpu_launches": 2 * blocks * args.steps,
@@ -716,6 +736,7 @@ def main():
                          "its ranks emulated on one GPU (one GPU each)")
     ap.add_argument("--splits", type=int, default=0, help="decode: KV splits per sequence (0 = suggested)")
     ap.add_argument("--ring-ranks", type=int, default=8, help="ring: ranks emulated on the one GPU")
+    ap.add_argument("--no-graph", action="store_true", help="ring: time eager launches only (no CUDA graph)")
     ap.add_argument("--dtype", choices=["bf16", "fp8"], default="bf16",
                     help="forward inputs: bf16, or E4M3 codes with per-tensor scales")
     args = ap.parse_args()

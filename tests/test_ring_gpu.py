@@ -95,3 +95,23 @@ def test_emulated_ring_full_size_sampled_rows(cuda_ok, name, world, heads):
           f"lse max-abs {worst['lse_max_abs']:.3e}  ({len(rows)} rows x {len(heads)} heads)")
     del q, k, v, out, lse
     torch.cuda.empty_cache()
+
+
+def test_emulated_ring_replays_from_a_cuda_graph(cuda_ok):
+    # The benchmark times the emulated ring step as a CUDA graph replay: the
+    # captured launches must give the eager step's bits, replay after replay.
+    q, k, v = (t.cuda() for t in make_qkv(1, 4, 2, 1024, 128, 21))
+    shares = ring.emulate_shares(q, k, v, 4)
+    eager = ring.run_emulated(shares, "causal")
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        captured = ring.run_emulated(shares, "causal")
+    for _ in range(3):
+        for t in (x for res in captured for pair in res for x in pair):
+            t.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        for (eo, el), (co, cl) in zip(eager, captured):
+            for a, b in zip(eo + el, co + cl):
+                assert torch.equal(a, b)
