@@ -408,7 +408,7 @@ def run_ours(args, w):
                             "8 chunks, copies overlapped with the kernels",
                     "ms_per_step": e2e_ms / e2e_steps},
         }
-        if not args.no_cpu_baseline:
+        if not args.no_cpu_baseline and world == 1:   # the host-core baseline is an N = 1 figure
             if fp8:
                 line["cpu_baseline"] = fp8_cpu_baseline(w, q, k, v, sq, sk, sv)
             else:
