@@ -119,7 +119,7 @@ def _ring_worker(rank, world, port, mask, queue):
 
 
 @pytest.mark.timeout(180)
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 4])
 def test_gloo_ranks_exchange_halves(world):
     ctx = mp.get_context("spawn")
     queue = ctx.Queue()
