@@ -92,11 +92,31 @@ def _no_subnormal(codes):
 
 _orig = O8.e4m3_to_float
 
+
+def _nan_saturates(codes):
+    val = _orig(codes)
+    c = np.asarray(codes, dtype=np.uint8)
+    return np.where(np.isnan(val), np.where(c & 0x80, -448.0, 448.0), val)
+
+
+def _k_takes_v_scale(q8, k8, v8, q_scale, k_scale, v_scale, scale=None, mask_kind=1, window=None, rows=None):
+    return F.attention(O8.dequantise(q8, q_scale), O8.dequantise(k8, v_scale), O8.dequantise(v8, v_scale),
+                       scale, mask_kind, window, rows=rows)
+
+
+def _softmax_scale_dropped(q8, k8, v8, q_scale, k_scale, v_scale, scale=None, mask_kind=1, window=None, rows=None):
+    return F.attention(O8.dequantise(q8, q_scale), O8.dequantise(k8, k_scale), O8.dequantise(v8, v_scale),
+                       None, mask_kind, window, rows=rows)
+
+
 MUTANTS = {
     "exponent bias 8": ("e4m3_to_float", _bias8),
     "subnormals read as normals": ("e4m3_to_float", _no_subnormal),
     "sign bit dropped": ("e4m3_to_float", lambda c: np.abs(_orig(c))),
+    "NaN codes saturate to 448": ("e4m3_to_float", _nan_saturates),
     "scale ignored": ("dequantise", lambda codes, scale: _orig(codes)),
+    "k dequantised with the v scale": ("attention_fp8", _k_takes_v_scale),
+    "softmax scale dropped": ("attention_fp8", _softmax_scale_dropped),
 }
 
 
