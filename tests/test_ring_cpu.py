@@ -119,12 +119,12 @@ def _ring_worker(rank, world, port, mask, queue):
 
 
 @pytest.mark.timeout(180)
-@pytest.mark.parametrize("world", [2, 3, 4])
-def test_gloo_ranks_exchange_halves(world):
+@pytest.mark.parametrize("world,mask", [(2, "causal"), (3, "causal"), (4, "causal"), (3, "full")])
+def test_gloo_ranks_exchange_halves(world, mask):
     ctx = mp.get_context("spawn")
     queue = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_ring_worker, args=(r, world, port, "causal", queue)) for r in range(world)]
+    procs = [ctx.Process(target=_ring_worker, args=(r, world, port, mask, queue)) for r in range(world)]
     for p in procs:
         p.start()
     got = sorted((queue.get(timeout=150) for _ in procs), key=lambda t: t[0])
@@ -134,6 +134,7 @@ def test_gloo_ranks_exchange_halves(world):
     out = ring.zigzag_gather([(torch.from_numpy(g[1]), torch.from_numpy(g[2])) for g in got]).numpy()
     lse = ring.zigzag_gather([(torch.from_numpy(g[3]), torch.from_numpy(g[4])) for g in got]).numpy()
     q, k, v = _inputs(1, 4, 2, 8 * world, 8, 77)
-    ref_o, ref_l = oracle.attention(q.numpy(), k.numpy(), v.numpy(), 1 / math.sqrt(8), 1)
+    ref_o, ref_l = oracle.attention(q.numpy(), k.numpy(), v.numpy(), 1 / math.sqrt(8),
+                                    {"full": 0, "causal": 1}[mask])
     assert np.abs(out - ref_o).max() < 1e-12
     assert np.abs(lse - ref_l).max() < 1e-12
