@@ -285,3 +285,21 @@ def test_host_forward_valid_arguments_reach_the_device(lib):
     assert call_host(lib, hq=HQ + 3, ho=HO + 2) == 4  # host buffers need no alignment
     assert call_host(lib, chunks=100) == 4
     assert call_host(lib, fp8=True, d=128) == 4
+
+
+def test_host_binding_validates_before_touching_a_device():
+    import torch
+    bf = dict(dtype=torch.bfloat16)
+    q, k = torch.zeros(1, 4, 8, 64, **bf), torch.zeros(1, 2, 8, 64, **bf)
+    with pytest.raises(ValueError):                       # v shaped unlike k
+        A.fwd_host(q, k, torch.zeros(1, 2, 9, 64, **bf))
+    with pytest.raises(ValueError):                       # wrong dtype
+        A.fwd_host(q.float(), k, k)
+    with pytest.raises(ValueError):                       # not contiguous
+        A.fwd_host(q.transpose(2, 3), k, k)
+    with pytest.raises(ValueError):                       # unknown mask
+        A.fwd_host(q, k, k, mask="banded")
+    with pytest.raises(ValueError):                       # outputs of the wrong shape
+        A.fwd_host(q, k, k, out=torch.zeros(1, 4, 8, 32, **bf))
+    with pytest.raises(ValueError):                       # FP8 codes must be uint8 / float8_e4m3fn
+        A.fwd_fp8_host(q, k, k, 1.0, 1.0, 1.0)
