@@ -97,6 +97,9 @@ int validate(const void* const ptrs[10], int64_t B, int64_t Hq, int64_t Hkv, int
   if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window < 1) return ATTN_ERR_INVALID_ARG;
   if (N > (int64_t(1) << 30) || B * Hq > (int64_t(1) << 30)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  // Byte counts below are int64 products: keep q's element count within 2^50.
+  if (static_cast<double>(B * Hq) * static_cast<double>(N) * static_cast<double>(d) > 1125899906842624.0)
+    return ATTN_ERR_INVALID_ARG;
   if (eb == 1 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (!std::isfinite(score_scale) || !(score_scale > 0.f) || !std::isfinite(v_scale) || !(v_scale > 0.f))
     return ATTN_ERR_INVALID_ARG;

@@ -303,3 +303,8 @@ def test_host_binding_validates_before_touching_a_device():
         A.fwd_host(q, k, k, out=torch.zeros(1, 4, 8, 32, **bf))
     with pytest.raises(ValueError):                       # FP8 codes must be uint8 / float8_e4m3fn
         A.fwd_fp8_host(q, k, k, 1.0, 1.0, 1.0)
+
+
+def test_host_forward_rejects_sizes_beyond_any_memory(lib):
+    # 2^30 rows of 2^20 heads x 128: far beyond any memory; refused before any product overflows
+    assert call_host(lib, B=1, Hq=1 << 20, Hkv=1 << 20, N=1 << 30, d=128) == 1
