@@ -145,8 +145,9 @@ int attn_fwd_fp8_ex(const void* q, const void* k, const void* v, float q_scale, 
  * not block the host unless the host memory is pageable, in which case the runtime may
  * copy synchronously. The library keeps two copy streams per device, created on first
  * use, and allocates no memory. Errors: arguments are checked before anything is
- * enqueued, as in attn_fwd. If a copy or launch fails part way, ATTN_ERR_CUDA is
- * returned; `stream` is still ordered after whatever had been enqueued.
+ * enqueued, as in attn_fwd. If something fails part way, its status is returned:
+ * ATTN_ERR_CUDA for a copy, the chunk's attn_fwd status for a launch (ATTN_ERR_UNSUPPORTED
+ * without an sm_100 device). `stream` is still ordered after whatever had been enqueued.
  */
 int attn_fwd_host(const void* hq, const void* hk, const void* hv, void* hout, float* hlse,
                   void* dq, void* dk, void* dv, void* dout, float* dlse,
