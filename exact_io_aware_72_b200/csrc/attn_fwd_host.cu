@@ -35,10 +35,15 @@ std::mutex g_copy_mutex;
 CopyStreams g_copy[kMaxDevices];
 
 // Two non-blocking copy streams per device, created on first use and kept.
+// An unsupported device is refused here, before anything is enqueued.
 int copy_streams(CopyStreams& out) {
-  int dev = 0;
+  int dev = 0, major = 0, minor = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (major != 10 || minor != 0) return ATTN_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_copy_mutex);
   CopyStreams& cs = g_copy[dev];
   if (!cs.up && cudaStreamCreateWithFlags(&cs.up, cudaStreamNonBlocking) != cudaSuccess) return ATTN_ERR_CUDA;

@@ -145,9 +145,10 @@ int attn_fwd_fp8_ex(const void* q, const void* k, const void* v, float q_scale, 
  * not block the host unless the host memory is pageable, in which case the runtime may
  * copy synchronously. The library keeps two copy streams per device, created on first
  * use, and allocates no memory. Errors: arguments are checked before anything is
- * enqueued, as in attn_fwd. If something fails part way, its status is returned:
- * ATTN_ERR_CUDA for a copy, the chunk's attn_fwd status for a launch (ATTN_ERR_UNSUPPORTED
- * without an sm_100 device). `stream` is still ordered after whatever had been enqueued.
+ * enqueued, as in attn_fwd, and so is the device (ATTN_ERR_UNSUPPORTED unless sm_100).
+ * If something fails part way, its status is returned: ATTN_ERR_CUDA for a copy, the
+ * chunk's attn_fwd status for a launch. `stream` is still ordered after whatever had been
+ * enqueued.
  */
 int attn_fwd_host(const void* hq, const void* hk, const void* hv, void* hout, float* hlse,
                   void* dq, void* dk, void* dv, void* dout, float* dlse,
