@@ -22,7 +22,7 @@ EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_status_string", "attn_debug_error", 
            "attn_bwd", "attn_bwd_ex", "attn_bwd_workspace_bytes", "attn_bwd_debug_error",
            "attn_decode", "attn_decode_ex", "attn_decode_workspace_bytes", "attn_decode_num_splits",
            "attn_decode_debug_error", "attn_fwd_fp8", "attn_fwd_fp8_ex", "attn_merge", "attn_fwd_host",
-           "attn_fwd_fp8_host")
+           "attn_fwd_fp8_host", "attn_decode_static")
 
 _lib = None
 
@@ -89,6 +89,8 @@ def load_library():
     lib.attn_decode_num_splits.restype = i64
     lib.attn_decode_debug_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.attn_decode_debug_error.restype = ctypes.c_int
+    lib.attn_decode_static.argtypes = [vp] * 7 + [i64] * 9 + [ctypes.c_float, ctypes.c_int, i64, vp]
+    lib.attn_decode_static.restype = ctypes.c_int
     host_tail = [vp] * 7 + [i64] * 5 + [f32, ctypes.c_int, i64, i64, vp]
     lib.attn_fwd_host.argtypes = [vp, vp, vp] + host_tail
     lib.attn_fwd_host.restype = ctypes.c_int
@@ -330,6 +332,49 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
                                 ctypes.c_void_p(stream.cuda_stream), ctypes.byref(opts))
     if st != 0:
         raise AttnError(st, "attn_decode")
+    return out, lse
+
+
+# Bytes of the library's own scratch array used by attn_decode_static (include/attn.h).
+DECODE_STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
+
+
+def decode_static(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_table: torch.Tensor,
+                  seq_lens: torch.Tensor, out: torch.Tensor, lse: torch.Tensor, num_splits: int,
+                  scale: Optional[float] = None, mask: str = "causal", window: Optional[int] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """``decode`` through ``attn_decode_static``: the library's fixed scratch array
+    instead of a workspace, for callers that hand over only their inputs and
+    outputs and cannot allocate device memory.  Nothing is allocated here either:
+    ``out`` (bf16 [B,Hq,Nq,d]) and ``lse`` (fp32 [B,Hq,Nq]) are the caller's, and
+    ``num_splits`` is explicit (it decides the scratch size, at most
+    DECODE_STATIC_SCRATCH_BYTES).  Calls that overlap on the GPU share the array
+    and race; keep them on one stream."""
+    lib = load_library()
+    for t, name, dt, nd in ((q, "q", torch.bfloat16, 4), (k_cache, "k_cache", torch.bfloat16, 4),
+                            (v_cache, "v_cache", torch.bfloat16, 4), (block_table, "block_table", torch.int32, 2),
+                            (seq_lens, "seq_lens", torch.int32, 1), (out, "out", torch.bfloat16, 4),
+                            (lse, "lse", torch.float32, 3)):
+        _check(t, name, dt, nd)
+    B, Hq, Nq, d = q.shape
+    num_pages, Hkv, page_size, dk = k_cache.shape
+    if dk != d or tuple(v_cache.shape) != tuple(k_cache.shape) or block_table.shape[0] != B \
+            or seq_lens.shape[0] != B or tuple(out.shape) != tuple(q.shape) or tuple(lse.shape) != (B, Hq, Nq):
+        raise ValueError("q, cache, block_table, seq_lens, out and lse shapes disagree")
+    if mask not in MASKS:
+        raise ValueError(f"mask must be one of {sorted(MASKS)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        st = lib.attn_decode_static(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
+                                    seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Nq, d,
+                                    num_pages, page_size, block_table.shape[1], int(num_splits), float(scale),
+                                    MASKS[mask], int(window) if window is not None else 0,
+                                    ctypes.c_void_p(stream.cuda_stream))
+    if st != 0:
+        raise AttnError(st, "attn_decode_static")
     return out, lse
 
 

@@ -324,3 +324,57 @@ extern "C" int attn_decode_debug_error(cudaStream_t stream, int* device_code) {
   if (code == 0) return ATTN_OK;
   return (code & (kDErrSeqLen | kDErrPage)) ? ATTN_ERR_INVALID_ARG : ATTN_ERR_TIMEOUT;
 }
+
+// ---------------------------------------------------------------- allocation-free variant
+// attn_decode_static (include/attn.h): the decoding step with its scratch -- the work
+// counter and the splits' partial results -- in this fixed device array instead of a
+// caller workspace, for callers that cannot allocate device memory. Every device that
+// loads the library holds the array until the process exits; all calls on a device
+// share it.
+static __device__ __align__(256) unsigned char g_dec_static_scratch[ATTN_DECODE_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_static_mutex;
+void* g_static_scratch_ptr[kMaxDevices];
+
+// Device address of the scratch array on the current device, looked up once per device.
+// In host code the array's name only stands in for it, so the address must come from the
+// runtime with the device current.
+int static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (!g_static_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_dec_static_scratch) != cudaSuccess || !ptr) return ATTN_ERR_CUDA;
+    g_static_scratch_ptr[dev] = ptr;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int attn_decode_static(const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* block_table, const int32_t* seq_lens, void* out, float* lse,
+                                  int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t d, int64_t num_pages,
+                                  int64_t page_size, int64_t max_pages_per_seq, int64_t num_splits, float scale,
+                                  int mask_kind, int64_t window, cudaStream_t stream) {
+  const size_t need = attn_decode_workspace_bytes(B, Hq, Nq, d, num_splits);
+  if (need == 0) return ATTN_ERR_INVALID_ARG;
+  if (need > sizeof(g_dec_static_scratch)) return ATTN_ERR_UNSUPPORTED;  // larger than the fixed array
+  DecDevice dev;
+  const int st = dec_device_setup(dev);  // refuses devices other than sm_100
+  if (st != ATTN_OK) return st;
+  void* scratch = nullptr;
+  const int sst = static_scratch_address(&scratch);
+  if (sst != ATTN_OK) return sst;
+  // The work counter must be zero when the kernel starts. A call that completes leaves it
+  // zero, but one that gave up on a wait may not, so every call clears it.
+  if (cudaMemsetAsync(scratch, 0, kSchedBytes, stream) != cudaSuccess) return ATTN_ERR_CUDA;
+  return attn_decode_ex(q, k_cache, v_cache, block_table, seq_lens, out, lse, scratch, sizeof(g_dec_static_scratch),
+                        B, Hq, Hkv, Nq, d, num_pages, page_size, max_pages_per_seq, num_splits, scale, mask_kind,
+                        window, stream, nullptr);
+}

@@ -318,6 +318,45 @@ int64_t attn_decode_num_splits(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, i
    that gave up, ATTN_ERR_INVALID_ARG for a bad sequence length or page-table entry. */
 int attn_decode_debug_error(cudaStream_t stream, int* device_code);
 
+/*
+ * attn_decode_static: attn_decode without a caller workspace, for callers that cannot
+ * allocate device memory. (The pages have no counterpart: this is a deployment variant
+ * of the decoding step above, with the same result.)
+ *
+ * Who needs it: code that runs inside a host program which owns all device memory and
+ * hands the code only its input and output buffers -- an inference-server plugin, an
+ * embedded runtime with a fixed memory plan, a language binding without a device
+ * allocator. There a cudaMalloc is either not permitted, breaks the owner's memory plan,
+ * or synchronises the device at a moment the caller does not control.
+ *
+ * Instead of `workspace`, the call uses a scratch array that the library itself defines
+ * in device memory: ATTN_DECODE_STATIC_SCRATCH_BYTES bytes, held by every GPU that loads
+ * the library until the process exits. Nothing is allocated by the call: no cudaMalloc,
+ * no cudaFree, no allocating library routine.
+ *
+ *   arguments    those of attn_decode without workspace and workspace_bytes, with the
+ *                same meaning, layouts, checks and errors
+ *   size limit   attn_decode_workspace_bytes(B, Hq, Nq, d, num_splits) must not exceed
+ *                ATTN_DECODE_STATIC_SCRATCH_BYTES; a larger step is refused with
+ *                ATTN_ERR_UNSUPPORTED before anything is enqueued (use fewer splits, a
+ *                smaller batch, or attn_decode with a workspace)
+ *
+ * Set-up: the first call on a device, with that device current, looks up the device
+ * address of the array (once per device); make that first call before any stream capture.
+ * Every call then enqueues, on `stream`, a clear of the array's work counter followed by
+ * the decoding launches. If attn_decode's argument checks then refuse the call, that
+ * clear, which touches only the library's own array, may already be enqueued.
+ * Every call on a device shares the one array, and the array keeps the last call's
+ * partial results: calls that overlap on the GPU (other streams, other host threads)
+ * race on it and give wrong results. Order them, e.g. on one stream.
+ */
+#define ATTN_DECODE_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
+int attn_decode_static(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                       const int32_t* seq_lens, void* out, float* lse,
+                       int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t d,
+                       int64_t num_pages, int64_t page_size, int64_t max_pages_per_seq, int64_t num_splits,
+                       float scale, int mask_kind, int64_t window, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
