@@ -19,9 +19,12 @@ bandwidth).  ``--dtype fp8`` runs the forward on E4M3 inputs (peak: the measured
 figure x 2).  ``--pass ring`` runs ring attention with all its ranks emulated on one GPU
 (``--ring-ranks R``).
 
-With --gpus N > 1 the script runs under torchrun, one rank per GPU; every rank
-runs its own shard of the global batch (weak scaling, no data-path collective)
-and rank 0 prints one JSON line with the max-over-ranks time.
+With --gpus N > 1 the script runs under torchrun, one rank per GPU, and rank 0
+prints one JSON line with the max-over-ranks time.  By default every rank runs
+its own shard of the global batch (weak scaling, no data-path collective);
+``--split heads`` instead splits the one workload's (batch, KV-group) units
+into contiguous ranges, one per rank (strong scaling, still no collective:
+``exact_io_aware_72_b200.shard``).
 """
 from __future__ import annotations
 
@@ -309,17 +312,28 @@ def run_ours(args, w):
     from exact_io_aware_72_b200 import fwd, fwd_fp8, fwd_fp8_host, fwd_host
     fp8 = args.dtype == "fp8"
 
-    # Each rank runs its own shard of the global batch: B sequences seeded by rank.
+    split_heads = args.split == "heads" and world > 1
+    # Each rank runs its own shard of the global batch: B sequences seeded by rank;
+    # or (--split heads) its contiguous range of the one workload's (b, KV-group) units.
+    seed = w.seed if split_heads else w.seed + 1000 * rank
     if fp8:
         from harness.inputs import make_qkv_fp8
-        (q, sq), (k, sk), (v, sv) = make_qkv_fp8(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed + 1000 * rank, device=device,
-                                                 sharp=w.sharp)
+        (q, sq), (k, sk), (v, sv) = make_qkv_fp8(w.B, w.Hq, w.Hkv, w.N, w.d, seed, device=device, sharp=w.sharp)
     else:
-        q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed + 1000 * rank, device=device, sharp=w.sharp)
+        q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, seed, device=device, sharp=w.sharp)
+    total_flops = workload_flops(w, w.B) * (1 if split_heads else world)
+    flops = workload_flops(w, w.B)   # this rank's work per step
+    units = None
+    if split_heads:
+        from exact_io_aware_72_b200 import shard
+        q, k, v, (u0, u1) = shard.head_shard(q, k, v, world, rank)
+        units = shard.shard_sizes(w.B, w.Hkv, world)
+        if q is None:
+            raise SystemExit(f"--split heads: rank {rank} has no (batch, KV-group) unit; use fewer GPUs")
+        flops = workload_flops(w, w.B) * (u1 - u0) // (w.B * w.Hkv)
     out = torch.empty(q.shape, dtype=torch.bfloat16, device=device)
-    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=device)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
-    flops = workload_flops(w, w.B)
 
     def step():
         if fp8:
@@ -391,16 +405,18 @@ def run_ours(args, w):
         avg_launch_s = statistics.mean(per_launch_ms) / 1e3
         achieved = flops / avg_launch_s / 1e12
         peak = float(peaks["bf16_tflops"]) * (FP8_OVER_BF16 if fp8 else 1.0)
-        value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+        value = total_flops * args.steps / (total_ms / 1e3) / 1e12
         traffic = NCU_TRAFFIC.get((w.name + ("_fp8" if fp8 else ""), kernel_hash()))
         line = {
             "metric": FP8_METRIC if fp8 else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
+            "higher_is_better": True, "scaling": "strong" if split_heads else "weak", "vs_baseline": None,
+            "dtype": "e4m3" if fp8 else "bf16",
             "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
                        "mask": w.mask, "window": w.window, "sharp_rows": w.sharp,
-                       "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"dp{world}",
+                       "global_batch": w.B if split_heads else w.B * world, "seq_len": w.N,
+                       "parallelism": f"heads{world}" if split_heads else f"dp{world}",
                        "l2": "inputs larger than L2 (no flush)"},
             "frac_of_peak": value / world / peak,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -412,12 +428,14 @@ def run_ours(args, w):
             "gpu_launches": args.steps,
             "launch_ms": {"median": statistics.median(per_launch_ms), "best": min(per_launch_ms)},
             "clocks": clk,
-            "e2e": {"value": world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": total_flops * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "path": ("attn_fwd_fp8_host" if fp8 else "attn_fwd_host") + " from pinned host memory, "
                             "8 chunks, copies overlapped with the kernels",
                     "ms_per_step": e2e_ms / e2e_steps},
         }
+        if units is not None:
+            line["config"]["units_per_rank"] = units
         if not args.no_cpu_baseline and world == 1:   # the host-core baseline is an N = 1 figure
             if fp8:
                 line["cpu_baseline"] = fp8_cpu_baseline(w, q, k, v, sq, sk, sv)
@@ -749,6 +767,9 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="ring: time eager launches only (no CUDA graph)")
     ap.add_argument("--dtype", choices=["bf16", "fp8"], default="bf16",
                     help="forward inputs: bf16, or E4M3 codes with per-tensor scales")
+    ap.add_argument("--split", choices=["batch", "heads"], default="batch",
+                    help="with N > 1 GPUs: every rank its own batch (weak scaling), or the workload's "
+                         "(batch, KV-group) units split across ranks (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
