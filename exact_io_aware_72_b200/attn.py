@@ -15,8 +15,9 @@ import torch
 
 MASKS = {"full": 0, "causal": 1, "sliding_window": 2}
 STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_MISALIGNED",
-          4: "ATTN_ERR_CUDA", 5: "ATTN_ERR_TIMEOUT"}
+          4: "ATTN_ERR_CUDA", 5: "ATTN_ERR_TIMEOUT", 6: "ATTN_ERR_RANGE"}
 ATTN_ERR_TIMEOUT = 5
+ATTN_ERR_RANGE = 6
 LIB_NAME = "libattn_b200.so"
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_status_string", "attn_debug_error", "attn_fwd_num_work_items",
            "attn_bwd", "attn_bwd_ex", "attn_bwd_workspace_bytes", "attn_bwd_debug_error",
@@ -34,8 +35,10 @@ class AttnError(RuntimeError):
 
 
 class FwdOptions(ctypes.Structure):
+    """attn_fwd_options of include/attn.h."""
     _fields_ = [("wait_timeout_ns", ctypes.c_uint64), ("inject_stall", ctypes.c_int),
-                ("grid_ctas", ctypes.c_int)]
+                ("grid_ctas", ctypes.c_int), ("item_visits", ctypes.c_void_p), ("p_bf16", ctypes.c_int),
+                ("out_fp32", ctypes.c_int)]
 
 
 def lib_path() -> str:
@@ -112,13 +115,17 @@ def _check(t: torch.Tensor, name: str, dtype, ndim):
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
         mask: str = "causal", window: Optional[int] = None, out: Optional[torch.Tensor] = None,
         lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
-        wait_timeout_ns: int = 0, inject_stall: bool = False, grid_ctas: int = 0
-        ) -> Tuple[torch.Tensor, torch.Tensor]:
+        wait_timeout_ns: int = 0, inject_stall: bool = False, grid_ctas: int = 0, p_bf16: bool = False,
+        item_visits: Optional[torch.Tensor] = None, out_fp32: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
     """Exact attention forward: returns (out bf16 [B,Hq,N,d], lse fp32 [B,Hq,N]).
 
     q: [B,Hq,N,d], k/v: [B,Hkv,N,d], bf16, contiguous, on one CUDA device.
     ``mask`` is "full", "causal" or "sliding_window" (keys i-window < j <= i).
     The launch is asynchronous on ``stream`` (default: the current stream).
+    ``p_bf16`` selects bf16 P for V values beyond the fp16 range (see
+    include/attn.h); ``item_visits`` (int32 CUDA tensor of num_work_items
+    counters) is a test hook counting each work item's visits; ``out_fp32``
+    returns out in fp32, unrounded (partial results to merge).
     """
     lib = load_library()
     _check(q, "q", torch.bfloat16, 4)
@@ -132,15 +139,22 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float
         raise ValueError(f"mask must be one of {sorted(MASKS)}")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    out_dtype = torch.float32 if out_fp32 else torch.bfloat16
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
-    _check(out, "out", torch.bfloat16, 4)
+    _check(out, "out", out_dtype, 4)
     _check(lse, "lse", torch.float32, 3)
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    opts = FwdOptions(int(wait_timeout_ns), 1 if inject_stall else 0, int(grid_ctas))
+    visits = None
+    if item_visits is not None:
+        if not (item_visits.is_cuda and item_visits.dtype == torch.int32 and item_visits.is_contiguous()):
+            raise ValueError("item_visits must be a contiguous int32 CUDA tensor")
+        visits = item_visits.data_ptr()
+    opts = FwdOptions(int(wait_timeout_ns), 1 if inject_stall else 0, int(grid_ctas), visits, 1 if p_bf16 else 0,
+                      1 if out_fp32 else 0)
     with torch.cuda.device(q.device):
         st = lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                              B, Hq, Hkv, N, d, float(scale), MASKS[mask],
@@ -275,7 +289,7 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
            mask: str = "causal", window: Optional[int] = None, num_splits: Optional[int] = None,
            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
            workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
-           wait_timeout_ns: int = 0, grid_ctas: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
+           wait_timeout_ns: int = 0, grid_ctas: int = 0, p_bf16: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
     """One decoding step against a paged KV cache: returns (out bf16 [B,Hq,Nq,d],
     lse fp32 [B,Hq,Nq]).
 
@@ -323,7 +337,7 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
     ws_ptr, ws_len = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    opts = FwdOptions(int(wait_timeout_ns), 0, int(grid_ctas))
+    opts = FwdOptions(int(wait_timeout_ns), 0, int(grid_ctas), None, 1 if p_bf16 else 0)
     with torch.cuda.device(q.device):
         st = lib.attn_decode_ex(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
                                 seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(), ws_ptr, ws_len,
@@ -380,13 +394,13 @@ def decode_static(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
 
 def merge(acc_out: torch.Tensor, acc_lse: torch.Tensor, part_out: torch.Tensor, part_lse: torch.Tensor,
           first: bool = False, out: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
-    """Fold a partial attention result (bf16 out, fp32 lse of one block of keys)
-    into an fp32 accumulator in place (``first``: set it instead); when ``out``
-    (bf16) is given the merged rows are also written there."""
+    """Fold a partial attention result (out bf16 or fp32, lse fp32 of one block of
+    keys) into an fp32 accumulator in place (``first``: set it instead); when
+    ``out`` (bf16) is given the merged rows are also written there."""
     lib = load_library()
-    if not (acc_out.dtype == torch.float32 and acc_lse.dtype == torch.float32 and part_out.dtype == torch.bfloat16
-            and part_lse.dtype == torch.float32):
-        raise ValueError("merge: acc fp32, part_out bf16, lse fp32")
+    if not (acc_out.dtype == torch.float32 and acc_lse.dtype == torch.float32 and
+            part_out.dtype in (torch.bfloat16, torch.float32) and part_lse.dtype == torch.float32):
+        raise ValueError("merge: acc fp32, part_out bf16 or fp32, lse fp32")
     for t, name in ((acc_out, "acc_out"), (acc_lse, "acc_lse"), (part_out, "part_out"), (part_lse, "part_lse")):
         if not (t.is_cuda and t.is_contiguous()):
             raise ValueError(f"{name} must be a contiguous CUDA tensor")
@@ -400,7 +414,8 @@ def merge(acc_out: torch.Tensor, acc_lse: torch.Tensor, part_out: torch.Tensor, 
         stream = torch.cuda.current_stream(acc_out.device)
     with torch.cuda.device(acc_out.device):
         st = lib.attn_merge(acc_out.data_ptr(), acc_lse.data_ptr(), part_out.data_ptr(), part_lse.data_ptr(),
-                            out.data_ptr() if out is not None else None, rows, d, 0 if first else 1,
+                            out.data_ptr() if out is not None else None, rows, d,
+                            (0 if first else 1) | (2 if part_out.dtype == torch.float32 else 0),
                             ctypes.c_void_p(stream.cuda_stream))
     if st != 0:
         raise AttnError(st, "attn_merge")
@@ -480,6 +495,10 @@ def _fwd_host(fp8: bool, q, k, v, q_scale, k_scale, v_scale, scale, mask, window
         else:
             st = lib.attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), *common)
     if st != 0:
+        # A failure part way may leave copies in flight that read or write the
+        # staging tensors; wait for them (the call keeps `stream` ordered after
+        # them) before those tensors can return to the allocator.
+        stream.synchronize()
         raise AttnError(st, "attn_fwd_fp8_host" if fp8 else "attn_fwd_host")
     stream.synchronize()
     return out, lse

@@ -122,7 +122,9 @@ cudaError_t launch_bwd(const BwdParams& p, int grid, cudaStream_t stream) {
 extern "C" {
 
 size_t attn_bwd_workspace_bytes(int64_t B, int64_t Hq, int64_t N) {
-  if (B < 1 || Hq < 1 || N < 1) return 0;
+  if (B < 1 || Hq < 1 || N < 1 || B > (int64_t(1) << 30) || Hq > (int64_t(1) << 30) || N > (int64_t(1) << 30) ||
+      B * Hq > (int64_t(1) << 61) / (N * 4))
+    return 0;
   return static_cast<size_t>(B) * static_cast<size_t>(Hq) * static_cast<size_t>(N) * sizeof(float);
 }
 
@@ -137,6 +139,8 @@ int attn_bwd_ex(const void* q, const void* k, const void* v, const void* out, co
   if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window < 1) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  // Byte counts must fit in 63 bits (B * Hq * N <= 2^60 after sizes_ok).
+  if (B * Hq * N > (int64_t(1) << 61) / (d * 4)) return ATTN_ERR_INVALID_ARG;
   const size_t ws = attn_bwd_workspace_bytes(B, Hq, N);
   if (workspace_bytes < ws) return ATTN_ERR_INVALID_ARG;
   const size_t q_bytes = static_cast<size_t>(B * Hq * N * d) * 2;

@@ -53,7 +53,7 @@ std::mutex g_dev_mutex;
 DeviceInfo g_dev[kMaxDevices];
 
 // Probe the current device once: sm_100 check, SM count, error-word address,
-// and the dynamic shared-memory opt-in of both kernel instances.
+// and the dynamic shared-memory opt-in of every kernel instance.
 int device_setup(int& dev, DeviceInfo& out_info) {
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
@@ -75,8 +75,12 @@ int device_setup(int& dev, DeviceInfo& out_info) {
                                SmemLayout<64>::kAlloc) != cudaSuccess ||
           cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SmemLayout<128>::kAlloc) != cudaSuccess ||
-          cudaFuncSetAttribute(attn_fwd_kernel<128, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               SmemLayout<128, 1>::kAlloc) != cudaSuccess)
+          cudaFuncSetAttribute(attn_fwd_kernel<128, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SmemLayout<128, 1>::kAlloc) != cudaSuccess ||
+          cudaFuncSetAttribute(attn_fwd_kernel<64, 2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SmemLayout<64>::kAlloc) != cudaSuccess ||
+          cudaFuncSetAttribute(attn_fwd_kernel<128, 2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SmemLayout<128>::kAlloc) != cudaSuccess)
         return ATTN_ERR_CUDA;
     }
     info.probed = true;
@@ -109,6 +113,9 @@ int check_sizes(int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d, int ma
   if (N > (int64_t(1) << 30) || B * Hq > (int64_t(1) << 30) || B * Hkv > (int64_t(1) << 30))
     return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  // Byte counts (at most 4 bytes per element) must fit in 63 bits; B * Hq * N is
+  // at most 2^60 after the checks above, so the product itself cannot wrap.
+  if (B * Hq * N > (int64_t(1) << 61) / (d * 4)) return ATTN_ERR_INVALID_ARG;
   plan.mask_kind = mask_kind;
   plan.window = window;
   // A window covering every earlier key is plain causal attention.
@@ -153,9 +160,10 @@ int fwd_launch(const void* q, const void* k, const void* v, void* out, float* ls
   if (eb == 1 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (!std::isfinite(score_scale) || !(score_scale > 0.f) || !std::isfinite(v_scale) || !(v_scale > 0.f))
     return ATTN_ERR_INVALID_ARG;
+  const bool out_f32 = opts && opts->out_fp32;
   const size_t q_bytes = static_cast<size_t>(B * Hq * N * d) * eb;
   const size_t kv_bytes = static_cast<size_t>(B * Hkv * N * d) * eb;
-  const size_t out_bytes = static_cast<size_t>(B * Hq * N * d) * 2;
+  const size_t out_bytes = static_cast<size_t>(B * Hq * N * d) * (out_f32 ? 4 : 2);
   const size_t lse_bytes = static_cast<size_t>(B * Hq * N) * 4;
   if (overlaps(out, out_bytes, q, q_bytes) || overlaps(out, out_bytes, k, kv_bytes) ||
       overlaps(out, out_bytes, v, kv_bytes) || overlaps(lse, lse_bytes, out, out_bytes) ||
@@ -179,7 +187,8 @@ int fwd_launch(const void* q, const void* k, const void* v, void* out, float* ls
       encode_bhnd(enc, &p.tm_k, k, B * Hkv, N, d, eb) != CUDA_SUCCESS ||
       encode_bhnd(enc, &p.tm_v, v, B * Hkv, N, d, eb) != CUDA_SUCCESS)
     return ATTN_ERR_CUDA;
-  p.out = static_cast<__nv_bfloat16*>(out);
+  p.out = out_f32 ? nullptr : static_cast<__nv_bfloat16*>(out);
+  p.out_f32 = out_f32 ? static_cast<float*>(out) : nullptr;
   p.lse = lse;
   p.err = info.err_word;
   p.B = static_cast<int>(B);
@@ -199,6 +208,8 @@ int fwd_launch(const void* q, const void* k, const void* v, void* out, float* ls
   p.timeout_ns = (opts && opts->wait_timeout_ns) ? opts->wait_timeout_ns : kDefaultTimeoutNs;
   p.inject_stall = (opts && opts->inject_stall) ? 1 : 0;
   p.out_v8 = (reinterpret_cast<uintptr_t>(out) % 32 == 0) ? 1 : 0;
+  p.item_visits = opts ? opts->item_visits : nullptr;
+  const bool p_bf16 = opts && opts->p_bf16;
 
   int grid = info.sm_count;
   if (opts && opts->grid_ctas > 0) grid = opts->grid_ctas;
@@ -211,13 +222,15 @@ int fwd_launch(const void* q, const void* k, const void* v, void* out, float* ls
   cudaError_t e;
   if (eb == 1) {
     cfg.dynamicSmemBytes = SmemLayout<128, 1>::kAlloc;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, 1>, p);
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, 1, false>, p);
   } else if (d == 128) {
     cfg.dynamicSmemBytes = SmemLayout<128>::kAlloc;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128>, p);
+    e = p_bf16 ? cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, 2, false>, p)
+               : cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, 2, true>, p);
   } else {
     cfg.dynamicSmemBytes = SmemLayout<64>::kAlloc;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<64>, p);
+    e = p_bf16 ? cudaLaunchKernelEx(&cfg, attn_fwd_kernel<64, 2, false>, p)
+               : cudaLaunchKernelEx(&cfg, attn_fwd_kernel<64, 2, true>, p);
   }
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -234,6 +247,7 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_MISALIGNED: return "ATTN_ERR_MISALIGNED";
     case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
     case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    case ATTN_ERR_RANGE: return "ATTN_ERR_RANGE";
     default: return "ATTN_ERR_UNKNOWN";
   }
 }
@@ -282,7 +296,8 @@ int attn_debug_error(cudaStream_t stream, int* device_code) {
     if (cudaMemcpyToSymbol(g_attn_error, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
   }
   if (device_code) *device_code = code;
-  return code ? ATTN_ERR_TIMEOUT : ATTN_OK;
+  if (code == 0) return ATTN_OK;
+  return (code & kErrRangeV) ? ATTN_ERR_RANGE : ATTN_ERR_TIMEOUT;
 }
 
 }  // extern "C"

@@ -119,6 +119,11 @@ int validate(const void* const ptrs[10], int64_t B, int64_t Hq, int64_t Hkv, int
   const void* const* dv = ptrs + 5;  // dq, dk, dv, dout, dlse
   if (outputs_overlap(dv[0], dv[1], dv[2], dv[3], dv[4], u) || outputs_overlap(h[0], h[1], h[2], h[3], h[4], u))
     return ATTN_ERR_INVALID_ARG;
+  // The uploads write the device staging inputs, so unlike attn_fwd's inputs
+  // (which may alias, e.g. k == v) they must not overlap one another.
+  const size_t nq = u.q * u.count, nkv = u.kv * u.count;
+  if (overlaps(dv[0], nq, dv[1], nkv) || overlaps(dv[0], nq, dv[2], nkv) || overlaps(dv[1], nkv, dv[2], nkv))
+    return ATTN_ERR_INVALID_ARG;
   for (int i = 0; i < 4; ++i)
     if (reinterpret_cast<uintptr_t>(dv[i]) & 15u) return ATTN_ERR_MISALIGNED;
   if (reinterpret_cast<uintptr_t>(dv[4]) & 3u) return ATTN_ERR_MISALIGNED;
@@ -145,18 +150,25 @@ int host_forward(const void* hq, const void* hk, const void* hv, void* hout, flo
   st = copy_streams(cs);
   if (st != ATTN_OK) return st;
   EventSet events;
-  cudaEvent_t start = events.make();
-  if (!start || cudaEventRecord(start, stream) != cudaSuccess) return ATTN_ERR_CUDA;
+  // The join's two events are made before anything is enqueued, so a join never
+  // lacks an event; if recording or waiting on them fails, both copy streams are
+  // synchronised instead, which orders their copies before anything `stream` runs later.
+  cudaEvent_t start = events.make(), join_up = events.make(), join_down = events.make();
+  if (!start || !join_up || !join_down) return ATTN_ERR_CUDA;
+  if (cudaEventRecord(start, stream) != cudaSuccess) return ATTN_ERR_CUDA;
   // Nothing is copied into the staging buffers before earlier work on `stream` is done.
   if (cudaStreamWaitEvent(cs.up, start, 0) != cudaSuccess || cudaStreamWaitEvent(cs.down, start, 0) != cudaSuccess)
     return ATTN_ERR_CUDA;
   // On every exit past this point `stream` waits for both copy streams, so that
   // whatever was enqueued is ordered before the caller's later work.
   auto join = [&](int status) -> int {
-    cudaEvent_t a = events.make(), b = events.make();
-    if (!a || !b || cudaEventRecord(a, cs.up) != cudaSuccess || cudaEventRecord(b, cs.down) != cudaSuccess ||
-        cudaStreamWaitEvent(stream, a, 0) != cudaSuccess || cudaStreamWaitEvent(stream, b, 0) != cudaSuccess)
+    if (cudaEventRecord(join_up, cs.up) != cudaSuccess || cudaEventRecord(join_down, cs.down) != cudaSuccess ||
+        cudaStreamWaitEvent(stream, join_up, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(stream, join_down, 0) != cudaSuccess) {
+      cudaStreamSynchronize(cs.up);
+      cudaStreamSynchronize(cs.down);
       return ATTN_ERR_CUDA;
+    }
     return status;
   };
   auto range = [&](int64_t c, int64_t& u0, int64_t& n) {

@@ -11,8 +11,9 @@
 //   warps 4-7   softmax for query tile 1
 //   warp  8     TMA loader: Q tiles once per work item, K/V tiles through a ring
 //   warps 9-10  tcgen05 issuers, one warp per query tile: S = Q K^T and
-//               O += P V; warp 9 also owns the TMEM allocation
-//   warp  11    idle
+//               O += P V; warp 9 also owns the TMEM allocation; with bf16
+//               inputs each also converts a quarter of every V tile to fp16
+//   warp  11    bf16 inputs: converts the other half of every V tile to fp16
 // Registers: launched at 168 per thread; the softmax warpgroups raise theirs to
 // 208 and the third warpgroup drops to 88 (2*128*208 + 128*88 = 384*168).
 // A work item is two 128-row query tiles that read the same K/V tiles: two query
@@ -21,7 +22,15 @@
 // tile work, the tensor core runs the other tile's matmuls.
 //
 // TMEM (512 columns x 128 lanes, fp32): S0 [0,128) S1 [128,256) O0 and O1 after
-// them.  P (bf16, two per column) overwrites the first 64 columns of its S tile.
+// them.  P (fp16 with bf16 inputs, two per column; E4M3 with FP8 inputs, four per
+// column) overwrites the first columns of its S tile.
+//
+// Precision (bf16 inputs): S = Q K^T is a bf16 product with fp32 accumulation;
+// the softmax weights P are rounded to fp16 (11 significant bits) and V is
+// converted to fp16 in shared memory for O += P V, so a row dominated by a few
+// keys keeps its output within about 2^-12 of their spread before the one bf16
+// rounding of out.  (bf16 P, 8 bits, is kept for V values beyond the fp16 range
+// by request: F16P = false.)
 //
 // Every mbarrier wait is bounded by a global-timer limit; a wait that gives up
 // records a code in the device error word and raises a CTA-wide abort flag, and
@@ -46,20 +55,24 @@ constexpr uint32_t kSoftmaxRegs = 208;
 constexpr uint32_t kOtherRegs = 88;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * 168, "register split exceeds launch");
 constexpr float kLn2 = 0.6931471805599453f;
-// The running max is only moved when a row's max grows by more than this many
-// powers of two; until then P may exceed 1 by up to 2^32.  bf16 P and fp32 sums
-// and accumulators carry that without loss (relative precision does not depend
-// on scale; a row sum stays below 2^32 * 2^17 keys = 2^49), and the final O / l
-// and log-sum-exp use the same max, so the result is unchanged.  A large margin
-// keeps O rescales (a TMEM round trip on the softmax critical path) rare even
-// for rows whose scores keep growing.
-constexpr float kRescaleThreshold = 32.0f;
-// P is packed to bf16 by truncating p * (1 + 2^-9): with the factor folded into
-// the exponent (x + log2(1 + 2^-9)), truncation lands within 3/4 of a bf16 ulp
-// of p (round-to-nearest would be 1/2) at the cost of one byte permute per pair.
-// The factor is common to every p of a row, so O / l is unaffected and the
-// log-sum-exp (from the fp32 sum) subtracts it exactly.
+// bf16 inputs: P goes to the tensor core as fp16 (11 significant bits, against
+// bf16's 8), so its rounding adds about 2^-12 relative per weight instead of 2^-9;
+// V is converted to fp16 in shared memory for the P V product (kind::f16 takes
+// one type for both operands).  The running max is only moved when a row's max
+// grows by more than kRescaleThresholdF16 powers of two, so P <= 2^15 < 65504, the
+// largest fp16 value; the final O / l and log-sum-exp use the same max, so the
+// result is unchanged, and the margin keeps O rescales (a TMEM round trip on the
+// softmax critical path) rare.
+constexpr float kRescaleThresholdF16 = 15.0f;
+// bf16 P (inputs with V beyond the fp16 range, by request): P is packed to bf16
+// by truncating p * (1 + 2^-9) -- with the factor folded into the exponent
+// (x + log2(1 + 2^-9)), truncation lands within 3/4 of a bf16 ulp of p at the
+// cost of one byte permute per pair -- and O is normalised by the sum of the
+// bf16 values written, so a row dominated by one key returns that key's v.  The
+// factor is common to every p of a row; the log-sum-exp (from the fp32 sum)
+// subtracts it.  The running max may lag the row max by up to 2^32 there.
 constexpr float kP16Bias = 0.0028150156f;  // log2(1 + 2^-9)
+constexpr float kRescaleThresholdBF16 = 32.0f;
 // E4M3 P (FP8 inputs): p is stored times 2^8, so weights down to 2^-14 of
 // the row max stay normal E4M3 numbers; the running max then moves whenever a
 // row's max grows by more than half a power of two (P <= 2^8.5 < 448, the
@@ -67,27 +80,20 @@ constexpr float kP16Bias = 0.0028150156f;  // log2(1 + 2^-9)
 // and the log-sum-exp subtracts it.
 constexpr float kP8Bias = 8.0f;
 constexpr float kRescaleThresholdE4M3 = 0.5f;
-// 2^f on [-1/2, 1/2]: degree-3 polynomial with minimal maximum relative error
-// (Remez exchange; csrc/fit_exp2_poly.py), max relative error 7.5e-5, used
-// after Cody-Waite reduction x = n + f for kPolyPairs of every 16 column pairs
-// so that part of the exponentials can run on the FMA pipe instead of the
-// MUFU.  Measured on B200 the softmax loop is bound by instruction issue, not
-// by the MUFU, so the offload is off (0 pairs); it pays only once the MUFU is
-// the limit.
-constexpr float kExp2Poly0 = 0.9999280572f;
-constexpr float kExp2Poly1 = 0.6932609677f;
-constexpr float kExp2Poly2 = 0.2426111251f;
-constexpr float kExp2Poly3 = 0.0551716685f;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + M rounds x to an integer in the low bits
-constexpr int kPolyPairs = 0;
+// V tiles converted to fp16 are signalled on a ring of this many barriers,
+// indexed by the K/V step (see softmax_role).
+constexpr int kConvRing = 4;
 // Steps before the end of a work item at which the loader prefetches the next
 // item's first tiles into L2 (each step is a few microseconds of work).
 constexpr int kPrefetchSteps = 6;
 
 enum : int { kMaskFull = 0, kMaskCausal = 1, kMaskWindow = 2 };
 
-// Error codes: role in bits 8..11, barrier index in bits 0..7.
-enum : int { kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3 };
+// Error codes: role in bits 8..11, barrier index in bits 0..7 for a wait that
+// gave up; kErrRangeV (with the KV head in the low bits) for a V value that
+// fp16 cannot hold.
+enum : int { kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3, kRoleVConv = 4 };
+constexpr int kErrRangeV = 1 << 20;
 
 struct FwdParams {
   CUtensorMap tm_q;  // [B*Hq, N, d] bf16, box 64 x 128, 128B swizzle
@@ -110,6 +116,8 @@ struct FwdParams {
   int inject_stall;
   int out_v8;        // 1: out is 32-byte aligned, rows are written with 32-byte stores
   float v_scale;     // FP8 inputs: the V tensor's scale, applied to O in the epilogue
+  unsigned int* item_visits;  // test hook: per work item, incremented once per visit (or null)
+  float* out_f32;    // non-null: out is written here in fp32 (partial results to merge) instead of bf16
 };
 
 // EB = bytes per input element: 2 for bf16, 1 for E4M3 (head dim 128 only).
@@ -134,7 +142,8 @@ struct SmemLayout {
   static constexpr int kOFree = kODone + 2;
   static constexpr int kFin = kOFree + 2;
   static constexpr int kTurn = kFin + 2;
-  static constexpr int kNumBars = kTurn + 2;
+  static constexpr int kVConv = kTurn + 2;  // V tile of a step converted to fp16 (bf16 inputs)
+  static constexpr int kNumBars = kVConv + kConvRing;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
@@ -305,6 +314,70 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// ------------------------------------------------------------ V to fp16
+// bf16 inputs: every V tile is converted to fp16 in place in shared memory for
+// the fp16 P V product (element-wise, so the swizzled layout does not matter).
+// Warp 11 converts the first half of each tile as soon as it lands; each MMA
+// warp converts a quarter of the NEXT step's tile right after issuing its S
+// product of a step, long before it next issues (after the softmax of its
+// tile), so neither tile's P V waits on the other tile's progress.  The three
+// arrive on kVConv[v % kConvRing] for K/V step v, and the P V of step v waits
+// there.  A barrier of the ring is reused four steps later; by then both MMA
+// warps have passed its previous phase, because V_{v+4} cannot land before the
+// P V of step v has released ring space.
+template <int D, int EB>
+struct VConvSplit {
+  static constexpr int kUnits = static_cast<int>(SmemLayout<D, EB>::kTileBytes / 16);  // 16-byte units
+  static constexpr int kWarp11 = kUnits / 2;                                      // [0, kUnits / 2)
+  static constexpr int kMma = kUnits / 4;                                          // then one quarter per MMA warp
+};
+
+// Units [u0, u0 + n) of the tile at tile_base, lane-strided: bf16 to fp16 in
+// place.  Returns the per-half maximum of |v| seen (bf16 bits).
+__device__ __forceinline__ uint32_t convert_v_units(uint32_t tile_base, int u0, int n, int lane) {
+  uint32_t mag = 0;
+#pragma unroll 4
+  for (int i = lane; i < n; i += 32) {
+    const uint32_t a = tile_base + static_cast<uint32_t>(u0 + i) * 16;
+    uint32_t x0, x1, x2, x3;
+    ld_shared_v4(a, x0, x1, x2, x3);
+    mag = max_u16x2(max_u16x2(mag, x0 & 0x7fff7fffu), max_u16x2(x1 & 0x7fff7fffu, x2 & 0x7fff7fffu));
+    mag = max_u16x2(mag, x3 & 0x7fff7fffu);
+    st_shared_v4(a, bf16x2_to_f16x2(x0), bf16x2_to_f16x2(x1), bf16x2_to_f16x2(x2), bf16x2_to_f16x2(x3));
+  }
+  return mag;
+}
+
+// After a warp's part of a tile: make it visible to the tensor core's (async)
+// proxy, record a magnitude of 2^16 or more (bf16 bits 0x4780 and up: beyond
+// the largest fp16 value, or not finite) as kErrRangeV, arrive.
+__device__ __forceinline__ void finish_v_part(uint32_t bar, uint32_t mag, int* err, int lane) {
+  fence_proxy_async_smem();
+  if (__any_sync(0xffffffffu, max(mag >> 16, mag & 0xffffu) >= 0x4780u) && lane == 0) atomicCAS(err, 0, kErrRangeV);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
+
+// Warp 11: the first half of every V tile of this CTA's work, in step order.
+template <int D, int EB>
+__device__ __forceinline__ void vconv_role(const FwdParams& p, uint32_t sbase, const Waiter& w, int lane) {
+  using L = SmemLayout<D, EB>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  uint32_t v = 0;  // K/V steps so far; V of step v is load 2v + 1
+  Schedule sched(p, blockIdx.x, gridDim.x);
+  int hu, r;
+  while (sched.next(hu, r)) {
+    const WorkItem it = decode_item(p, hu, r);
+    for (int j = it.lo_u; j <= it.hi_u; ++j, ++v) {
+      const uint32_t vn = 2 * v + 1, slot = vn % L::kStages;
+      const bool got = w.wait(bar(L::kKVFull + slot), (vn / L::kStages) & 1, (kRoleVConv << 8) | (L::kKVFull + slot));
+      if (!__all_sync(0xffffffffu, got)) return;
+      const uint32_t mag = convert_v_units(sbase + L::kKVOff + slot * L::kTileBytes, 0, VConvSplit<D, EB>::kWarp11, lane);
+      finish_v_part(bar(L::kVConv + (v % kConvRing)), mag, w.err, lane);
+    }
+  }
+}
+
 // ------------------------------------------------------------ roles
 // L2 prefetch of the next work item's Q tiles and of its first two K/V tiles
 // (sched has already moved past the current item).
@@ -347,6 +420,7 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sbase
   int hu, r;
   while (ok && sched.next(hu, r)) {
     const WorkItem it = decode_item(p, hu, r);
+    if (p.item_visits) atomicAdd(p.item_visits + static_cast<size_t>(hu) * p.row_units + r, 1u);
     // Q of this item goes into the single Q buffer once the previous item's
     // last S has read it.  The item's first K and V tiles are issued before
     // that wait (their ring slots free up earlier), so they are already in
@@ -413,7 +487,7 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sbase
 //   S_t  = Q_t K_j^T          (after that P V in issue order, since P aliases S)
 // and releases K_j / V_{j-1} / Q with commits; the other tile's warp does the
 // same, so each ring slot is freed after both warps' reads complete.
-template <int D, int EB>
+template <int D, int EB, bool F16P>
 __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t tmem, const Waiter& w,
                                          int t) {
   using L = SmemLayout<D, EB>;
@@ -422,7 +496,10 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
   // product takes 32 bytes of K per row: 16 bf16 or 32 E4M3 elements.
   constexpr uint32_t idesc_s =
       EB == 2 ? idesc_bf16_f32(kBlockM, kBlockN, false) : idesc_e4m3_f32(kBlockM, kBlockN, false);
-  constexpr uint32_t idesc_o = EB == 2 ? idesc_bf16_f32(kBlockM, D, true) : idesc_e4m3_f32(kBlockM, D, true);
+  // P V: fp16 P and the fp16 copy of V, bf16 both, or E4M3 both.
+  constexpr bool kConvV = EB == 2 && F16P;
+  constexpr uint32_t idesc_o = EB == 1 ? idesc_e4m3_f32(kBlockM, D, true)
+                                       : (F16P ? idesc_f16_f32(kBlockM, D, true) : idesc_bf16_f32(kBlockM, D, true));
   constexpr int kKeysPerPv = 32 / EB;  // keys per P V product
   const uint32_t s_tmem = tmem + (t ? L::kSCol1 : L::kSCol0);
   const uint32_t o_tmem = tmem + (t ? L::kOCol1 : L::kOCol0);
@@ -439,14 +516,36 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
     return __all_sync(0xffffffffu, got);
   };
 
+  // This warp's quarter of the V tile of K/V step v (load 2v + 1) to fp16.
+  auto convert_quarter = [&](uint32_t v) -> bool {
+    const uint32_t vn = 2 * v + 1, vslot = vn % L::kStages;
+    if (!wait_all(bar(L::kKVFull + vslot), (vn / L::kStages) & 1, code | (L::kKVFull + vslot))) return false;
+    const uint32_t mag = convert_v_units(sbase + L::kKVOff + vslot * L::kTileBytes,
+                                         VConvSplit<D, EB>::kWarp11 + t * VConvSplit<D, EB>::kMma,
+                                         VConvSplit<D, EB>::kMma, threadIdx.x & 31);
+    finish_v_part(bar(L::kVConv + (v % kConvRing)), mag, w.err, threadIdx.x & 31);
+    return true;
+  };
+
   uint32_t kv_n = 0;
   uint32_t p_cnt = 0;
   int items = 0;
   bool ok = true;
   Schedule sched(p, blockIdx.x, gridDim.x);
+  if constexpr (kConvV) {
+    Schedule peek = sched;
+    int h0, r0;
+    if (peek.next(h0, r0)) ok = convert_quarter(0);
+  }
   int hu, r;
   while (ok && sched.next(hu, r)) {
     const WorkItem it = decode_item(p, hu, r);
+    bool more_items = false;  // a step follows this item's last one
+    if constexpr (kConvV) {
+      Schedule peek = sched;
+      int h2, r2;
+      more_items = peek.next(h2, r2);
+    }
     const int valid = t ? it.valid[1] : it.valid[0];
     const int lo = t ? it.lo[1] : it.lo[0];
     const int hi = t ? it.hi[1] : it.hi[0];
@@ -469,6 +568,12 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
       ++p_cnt;
       const uint32_t vslot = vn % L::kStages;
       if (!wait_all(bar(L::kKVFull + vslot), (vn / L::kStages) & 1, code | (L::kKVFull + vslot))) return false;
+      if constexpr (kConvV) {
+        // Warp 11 and both MMA warps have converted this V tile (K/V step vn / 2) to fp16.
+        const uint32_t v = vn >> 1;
+        if (!wait_all(bar(L::kVConv + (v % kConvRing)), (v / kConvRing) & 1, code | (L::kVConv + (v % kConvRing))))
+          return false;
+      }
       tc_fence_after_sync();
       const uint64_t vd = v_desc0 + ((vslot * L::kTileBytes) >> 4);
 #pragma unroll
@@ -477,7 +582,7 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
         // tile; their P is the next 8 TMEM columns (32 bytes per row).
         const uint64_t vk = vd + ((kk * kKeysPerPv * 128) >> 4);
         if constexpr (EB == 2)
-          mma_bf16_ts_elect(o_tmem, s_tmem + kk * 8, vk, idesc_o, (kk > 0 || !first_pv) ? 1u : 0u);
+          mma_bf16_ts_elect(o_tmem, s_tmem + kk * 8, vk, idesc_o, (kk > 0 || !first_pv) ? 1u : 0u);  // kind::f16
         else
           mma_e4m3_ts_elect(o_tmem, s_tmem + kk * 8, vk, idesc_o, (kk > 0 || !first_pv) ? 1u : 0u);
       }
@@ -528,6 +633,13 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
       if (j > it.lo_u) tc_commit_elect(bar(L::kKVEmpty + (kv_n - 1) % L::kStages));  // V_{j-1} read
       tc_commit_elect(bar(L::kKVEmpty + kslot));                                   // K_j read
       if (j == it.hi_u) tc_commit_elect(bar(L::kQEmpty));                          // Q read
+      if constexpr (kConvV) {
+        // This warp's quarter of the next step's V (its P V comes a step later).
+        if ((j < it.hi_u || more_items) && !convert_quarter((kv_n >> 1) + 1)) {
+          ok = false;
+          break;
+        }
+      }
       kv_n += 2;
     }
     if (!ok) break;
@@ -542,12 +654,13 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
   w.drain(bar(L::kFin + t), 0, code | (L::kFin + t));
 }
 
-template <int D, int EB>
+// Eight softmax warps, one thread per query row of their tile.
+template <int D, int EB, bool F16P>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase, uint32_t tmem,
                                              const Waiter& w, int warp, int lane) {
   using L = SmemLayout<D, EB>;
-  constexpr float kBias = EB == 2 ? kP16Bias : kP8Bias;
-  constexpr float kThreshold = EB == 2 ? kRescaleThreshold : kRescaleThresholdE4M3;
+  constexpr float kBias = EB == 1 ? kP8Bias : (F16P ? 0.f : kP16Bias);
+  constexpr float kThreshold = EB == 1 ? kRescaleThresholdE4M3 : (F16P ? kRescaleThresholdF16 : kRescaleThresholdBF16);
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
   const int t = warp >> 2;
   const int quarter = warp & 3;
@@ -573,8 +686,8 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
     const int hi = t ? it.hi[1] : it.hi[0];
     const int row = mblk * kBlockM + row_in_tile;
     float m_run = -INFINITY;
-    float l_run = 0.f;   // row sum of P as written (bf16), normalises O
-    float l_lse = 0.f;   // fp32 row sum of p (carries the kP16Bias factor)
+    float l_run = 0.f;   // row sum that normalises O (bf16 P: of the bf16 values written)
+    float l_lse = 0.f;   // fp32 row sum of p: the log-sum-exp (and O's normaliser otherwise)
     // Both softmax warpgroups walk the item's whole KV range so they can hand
     // the turn token back and forth: the exp loop of one tile runs while
     // the tensor core works on the other tile (the exp unit is the shared
@@ -632,50 +745,28 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
         ++turn_cnt;
       }
       if (active) {
-        // p = 2^(s*c - m) on column pairs (packed fp32 FMA); the first
-        // kPolyPairs pairs of every 16 use the polynomial on the FMA pipe, the
-        // rest the MUFU ex2.  P goes to TMEM 16 columns at a time.  O is
-        // normalised by the sum of exactly the bf16 values written (so a row
-        // dominated by one key returns that key's v); the log-sum-exp uses the
-        // fp32 sum of p.
+        // p = 2^(s*c - m) on column pairs (packed fp32 FMA, MUFU ex2), rounded to
+        // fp16 or bf16 (bf16 inputs) or E4M3 (FP8 inputs) and written to TMEM
+        // over the first columns of the S tile.  The fp32 sum of p gives the
+        // log-sum-exp and, except with bf16 P, normalises O.
         const uint64_t c2 = f32x2_pack(c, c);
         const uint64_t nb2 = f32x2_pack(neg_base + kBias, neg_base + kBias);
-        const uint64_t magic2 = f32x2_pack(kRoundMagic, kRoundMagic);
-        const uint64_t nmagic2 = f32x2_pack(-kRoundMagic, -kRoundMagic);
-        const uint64_t neg1 = f32x2_pack(-1.f, -1.f);
-        const uint64_t q3 = f32x2_pack(kExp2Poly3, kExp2Poly3), q2 = f32x2_pack(kExp2Poly2, kExp2Poly2);
-        const uint64_t q1 = f32x2_pack(kExp2Poly1, kExp2Poly1), q0 = f32x2_pack(kExp2Poly0, kExp2Poly0);
-        uint64_t so2 = 0, sl2 = 0;  // (+0.f, +0.f)
+        uint64_t sl2 = 0, so2 = 0;  // (+0.f, +0.f)
 #pragma unroll
         for (int chunk = 0; chunk < 4; ++chunk) {
-          uint32_t pk[EB == 2 ? 16 : 8];   // P columns: two bf16 or four E4M3 values each
+          uint32_t pk[EB == 2 ? 16 : 8];   // P columns: two fp16 or four E4M3 values each
           float prev0 = 0.f, prev1 = 0.f;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int e = chunk * 32 + 2 * i;
             const uint64_t x2 = f32x2_fma(f32x2_pack(s[e], s[e + 1]), c2, nb2);
-            float x0, x1, p0, p1;
+            float x0, x1;
             f32x2_unpack(x2, x0, x1);
-            if (i < kPolyPairs) {
-              // 2^x = 2^n q(f): n = round(x) via the magic constant, f = x - n,
-              // q by Horner, n added to the exponent field.  x is clamped at
-              // -125 so masked (-inf) entries give 2^-125 q(f), not garbage.
-              const uint64_t xc = f32x2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-              const uint64_t t2 = f32x2_add(xc, magic2);
-              const uint64_t f2 = f32x2_fma(f32x2_add(t2, nmagic2), neg1, xc);
-              uint64_t r2 = f32x2_fma(f2, q3, q2);
-              r2 = f32x2_fma(f2, r2, q1);
-              r2 = f32x2_fma(f2, r2, q0);
-              float r0, r1, t0, t1;
-              f32x2_unpack(r2, r0, r1);
-              f32x2_unpack(t2, t0, t1);
-              p0 = __uint_as_float(__float_as_uint(r0) + (__float_as_uint(t0) << 23));
-              p1 = __uint_as_float(__float_as_uint(r1) + (__float_as_uint(t1) << 23));
-            } else {
-              p0 = fast_exp2(x0);
-              p1 = fast_exp2(x1);
-            }
-            if constexpr (EB == 2) {
+            const float p0 = fast_exp2(x0);
+            const float p1 = fast_exp2(x1);
+            if constexpr (EB == 2 && F16P) {
+              pk[i] = pack_f16x2(p0, p1);  // round to nearest even
+            } else if constexpr (EB == 2) {
               pk[i] = __byte_perm(__float_as_uint(p0), __float_as_uint(p1), 0x7632);  // truncate to bf16x2
               so2 = f32x2_add(so2, f32x2_pack(__uint_as_float(__float_as_uint(p0) & 0xffff0000u),
                                               __uint_as_float(__float_as_uint(p1) & 0xffff0000u)));
@@ -695,12 +786,16 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
           else
             tmem_store_8cols(tS + chunk * 8, pk);
         }
-        if constexpr (EB == 1) so2 = sl2;  // E4M3: O is normalised by the fp32 sum of p
-        float so_lo, so_hi, sl_lo, sl_hi;
-        f32x2_unpack(so2, so_lo, so_hi);
+        float sl_lo, sl_hi;
         f32x2_unpack(sl2, sl_lo, sl_hi);
-        l_run = l_run * alpha + (so_lo + so_hi);
         l_lse = l_lse * alpha + (sl_lo + sl_hi);
+        if constexpr (EB == 2 && !F16P) {
+          float so_lo, so_hi;
+          f32x2_unpack(so2, so_lo, so_hi);
+          l_run = l_run * alpha + (so_lo + so_hi);
+        } else {
+          l_run = l_lse;
+        }
       }
       if (!active) {
         __syncwarp();
@@ -734,7 +829,25 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
     bool got = w.wait(bar(L::kODone + t), items & 1, (kRoleSoftmax << 8) | (L::kODone + t));
     if (!__all_sync(0xffffffffu, got)) break;
     tc_fence_after_sync();
-    if (valid) {
+    if (valid && p.out_f32) {
+      // fp32 out: O / l written unrounded, 128 bytes per 32 columns.
+      const bool row_ok = row < p.N;
+      const float inv_l = (l_run > 0.f) ? (EB == 2 ? 1.f : p.v_scale) / l_run : 0.f;
+      const size_t head_row = (static_cast<size_t>(it.b) * p.Hq + head) * p.N + (row_ok ? row : 0);
+      float4* dstf = reinterpret_cast<float4*>(p.out_f32 + head_row * D);
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_load_32cols(tO + cc * 32, o);
+        if (row_ok) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dstf[cc * 8 + v] = make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                                           __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+        }
+      }
+      if (row_ok) p.lse[head_row] = (m_run + __log2f(l_lse) - kBias) * kLn2;
+    } else if (valid) {
       const bool row_ok = row < p.N;
       const float inv_l = (l_run > 0.f) ? (EB == 2 ? 1.f : p.v_scale) / l_run : 0.f;
       const size_t head_row = (static_cast<size_t>(it.b) * p.Hq + head) * p.N + (row_ok ? row : 0);
@@ -776,7 +889,9 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
   tmem_store_wait();
 }
 
-template <int D, int EB = 2>
+// EB = bytes per input element (2: bf16, 1: E4M3); F16P (bf16 inputs): P and V
+// go to the P V product as fp16 (true) or as bf16 (false).
+template <int D, int EB = 2, bool F16P = true>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
   using L = SmemLayout<D, EB>;
   extern __shared__ uint8_t smem_raw[];
@@ -803,6 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       mbar_init(bar(L::kFin + t), 1);
       mbar_init(bar(L::kTurn + t), 4);         // one arrival per warp of the other warpgroup
     }
+    for (int i = 0; i < kConvRing; ++i) mbar_init(bar(L::kVConv + i), 3);  // warp 11 and both MMA warps
     for (int i = 0; i < 4; ++i) mbar_arrive(bar(L::kTurn + 0));  // tile 0 starts with the turn
     *abort_flag = 0;
     fence_mbar_init();
@@ -820,7 +936,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
   if (warp < 8) {
     reg_alloc_raise<kSoftmaxRegs>();
-    softmax_role<D, EB>(p, sbase, tmem, w, warp, lane);
+    softmax_role<D, EB, F16P>(p, sbase, tmem, w, warp, lane);
   } else {
     reg_alloc_lower<kOtherRegs>();
   }
@@ -828,7 +944,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     if (lane == 0) producer_role<D, EB>(p, sbase, w);
     __syncwarp();
   } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
-    mma_role<D, EB>(p, sbase, tmem, w, warp - kMmaWarp);
+    mma_role<D, EB, F16P>(p, sbase, tmem, w, warp - kMmaWarp);
+  } else if (warp == kMmaWarp + 2) {
+    if constexpr (EB == 2 && F16P) vconv_role<D, EB>(p, sbase, w, lane);
   }
 
   tc_fence_before_sync();

@@ -198,6 +198,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
          | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
 }
 
+// Instruction descriptor of kind::f16 with fp16 A and B (format code 0), fp32
+// accumulator, A K-major, B K-major or MN-major.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major) {
+  return (1u << 4)                               // D format: f32
+         | (0u << 7)                             // A format: f16
+         | (0u << 10)                            // B format: f16
+         | ((b_mn_major ? 1u : 0u) << 16)        // B major-ness
+         | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
+}
+
 // Instruction descriptor of kind::f8f6f4: E4M3 A and B (format code 0), fp32
 // accumulator, A K-major; B K-major or MN-major (MN-major is valid for E4M3).
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool b_mn_major) {
@@ -305,6 +316,42 @@ __device__ __forceinline__ void st_global_v8(void* ptr, uint32_t a, uint32_t b, 
   asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(a), "r"(b), "r"(c), "r"(d),
                "r"(e), "r"(f), "r"(g), "r"(h)
                : "memory");
+}
+
+// Two fp32 values to fp16 with round-to-nearest-even, lo in bits 0..15.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two bf16 values (one 32-bit word, element 0 in bits 0..15) to two fp16 values in
+// the same positions, rounding to nearest even.  Exact for magnitudes in
+// [2^-17, 65280]; larger finite magnitudes become infinities and smaller ones lose
+// low bits (fp16 subnormals).  The bf16 halves are widened to fp32 by byte moves.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  uint32_t r;
+  asm("{\n\t.reg .b32 lo, hi;\n\t"
+      "prmt.b32 lo, %1, 0, 0x1044;\n\t"
+      "and.b32 hi, %1, 0xffff0000;\n\t"
+      "cvt.rn.f16x2.f32 %0, hi, lo;\n\t}"
+      : "=r"(r)
+      : "r"(w));
+  return r;
+}
+
+// Per 16-bit half maximum of two unsigned words.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 // Packed fp32 pairs (sm_100): one instruction operates on two floats.

@@ -14,8 +14,9 @@ from rank r-1 (NCCL send/recv into local buffers, overlapped with the work).
 For each (query half i, key half j) block the sm_100a forward kernel computes
 a partial result with the block's own mask -- causal: every key of half j < i
 is visible ("full"), j == i is the causal diagonal, j > i is skipped; full:
-every block -- and ``attn_merge`` folds it into an fp32 accumulator by its
-log-sum-exp.  The merged rows equal the exact attention of the whole sequence.
+every block -- written in fp32, and ``attn_merge`` folds it into an fp32
+accumulator by its log-sum-exp; only the final merged rows are rounded to
+bf16.  The merged rows equal the exact attention of the whole sequence.
 
 Only the data movement and the loop live here; every arithmetic step runs in
 the library's CUDA kernels (``fwd`` and ``merge``).  ``local_attention`` and
@@ -67,8 +68,9 @@ def block_mask(qi: int, kj: int, mask: str) -> Optional[str]:
 
 
 def _default_local(q, k, v, mask, scale):
+    # Block results stay fp32 (unrounded) until the last merge rounds out to bf16 once.
     from .attn import fwd
-    return fwd(q, k, v, scale=scale, mask=mask)
+    return fwd(q, k, v, scale=scale, mask=mask, out_fp32=True)
 
 
 def _default_merge(acc_o, acc_l, part_o, part_l, first, out):

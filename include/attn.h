@@ -52,7 +52,9 @@ typedef enum {
   ATTN_ERR_UNSUPPORTED = 2,  /* head dimension other than 64 or 128, or no sm_100 device */
   ATTN_ERR_MISALIGNED = 3,   /* q, k, v or out not 16-byte aligned, lse not 4-byte aligned */
   ATTN_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed (launch, tensor-map encode) */
-  ATTN_ERR_TIMEOUT = 5       /* a device-side wait gave up (reported by attn_debug_error) */
+  ATTN_ERR_TIMEOUT = 5,      /* a device-side wait gave up (reported by attn_debug_error) */
+  ATTN_ERR_RANGE = 6         /* a V value that fp16 cannot hold (magnitude >= 2^16, or not finite) met
+                                the default fp16 P V product (reported by attn_debug_error) */
 } attn_status;
 
 /*
@@ -73,6 +75,13 @@ typedef enum {
  * Ownership: the caller owns every buffer. The library allocates no device memory and
  * never synchronises; out and lse are written by the kernel when the stream reaches it.
  * out and lse must not overlap each other or the inputs (ATTN_ERR_INVALID_ARG).
+ * Precision: scores and sums are fp32; the softmax weights P go to the tensor core as
+ * fp16 (11 significant bits), with V converted to fp16 on chip, and out is rounded once
+ * to bf16. V values must therefore have magnitude below 2^16 (every finite bf16 value
+ * up to 65280 qualifies); a larger or non-finite V value makes the launch's result
+ * undefined and is reported by attn_debug_error as ATTN_ERR_RANGE. attn_fwd_ex with
+ * p_bf16 = 1 takes any V, with P rounded to bf16 instead (8 significant bits: out can
+ * then be off by about one bf16 ulp of a value near 1 where one or two keys dominate).
  * Errors: every argument is checked before anything is enqueued; on error nothing is
  * launched and the status says why. ATTN_ERR_CUDA reports a failed launch. Device-side
  * waits are bounded (about 2 s); a wait that gives up makes the kernel stop early and
@@ -82,13 +91,22 @@ int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
              int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
              float scale, int mask_kind, int64_t window, cudaStream_t stream);
 
-/* Options for attn_fwd_ex. Zero-initialise, then set what is needed. */
+/* Options for attn_fwd_ex (and the _ex forms of the other calls, which say which
+   fields they read). Zero-initialise, then set what is needed. */
 typedef struct {
   uint64_t wait_timeout_ns; /* bound of every device-side wait; 0 = default (2 s) */
   int inject_stall;         /* test hook: 1 = the loader issues no copies, so every consumer
                                wait runs out and the kernel exits with ATTN_ERR_TIMEOUT
                                pending in attn_debug_error; nothing faults or hangs */
   int grid_ctas;            /* number of persistent CTAs; 0 = one per SM */
+  unsigned int* item_visits; /* test hook (forward): NULL, or a device array of
+                               attn_fwd_num_work_items() counters, each incremented once
+                               per visit of its work item (the caller zeroes it) */
+  int p_bf16;               /* 1 = P and V go to the P V product as bf16 (any V value, coarser
+                               P); 0 = fp16 (default; |V| below 2^16). bf16 inputs only */
+  int out_fp32;             /* forward: 1 = out is fp32 [B, Hq, N, d] (16-byte aligned) and
+                               receives O / l unrounded, for partial results that are merged
+                               afterwards (attn_merge mode 2 or 3); 0 = bf16 out */
 } attn_fwd_options;
 
 /* attn_fwd with options (same arguments, same checks); opts may be NULL. */
@@ -135,7 +153,9 @@ int attn_fwd_fp8_ex(const void* q, const void* k, const void* v, float q_scale, 
  *   hout, hlse    host pointers, layouts of attn_fwd's out and lse; must not overlap the
  *                 host inputs or each other
  *   dq, dk, dv, dout, dlse   device staging buffers with attn_fwd's sizes, alignment and
- *                 overlap rules (owned by the caller; their contents are overwritten)
+ *                 overlap rules (owned by the caller; their contents are overwritten);
+ *                 since the uploads write dq, dk and dv, these three must not overlap
+ *                 one another either (ATTN_ERR_INVALID_ARG)
  *   B ... window  as attn_fwd
  *   chunks        number of ranges, >= 0; 0 = 8; more than B * Hkv means B * Hkv
  *   stream        CUDA stream of the current device
@@ -172,12 +192,14 @@ int attn_fwd_fp8_host(const void* hq, const void* hk, const void* hv,
  *
  *   acc_out   device, fp32 [rows, d], 16-byte aligned; read (mode 1) and written
  *   acc_lse   device, fp32 [rows], natural log; read (mode 1) and written
- *   part_out  device, bf16 [rows, d] (attn_fwd's out for one block of keys), 8-byte aligned
+ *   part_out  device, [rows, d] (attn_fwd's out for one block of keys): bf16, 8-byte aligned
+ *             (modes 0, 1), or fp32, 16-byte aligned (modes 2, 3: attn_fwd_ex with out_fp32)
  *   part_lse  device, fp32 [rows] (attn_fwd's lse for the same block)
  *   out       device, bf16 [rows, d], 8-byte aligned, or NULL: when given, the merged rows are
  *             also written here rounded to bf16 (it may be part_out itself)
  *   rows      1 .. 2^33; d in {64, 128}
- *   mode      0: the accumulator is set to the partial; 1: the partial is merged into it
+ *   mode      0: the accumulator is set to the partial; 1: the partial is merged into it;
+ *             2, 3: the same with an fp32 partial (no bf16 rounding before the merge)
  * Errors as attn_fwd; nothing is allocated and nothing synchronises.
  */
 int attn_merge(float* acc_out, float* acc_lse, const void* part_out, const float* part_lse, void* out,
@@ -189,8 +211,13 @@ const char* attn_status_string(int status);
  * attn_debug_error: synchronise `stream`, read and clear the device error word of the
  * current device. Returns ATTN_OK if no device wait gave up since the last call,
  * ATTN_ERR_TIMEOUT if one did (the raw code, which names the waiting role, goes to
- * *device_code when device_code is not NULL), ATTN_ERR_CUDA if the synchronisation
- * itself failed.
+ * *device_code when device_code is not NULL), ATTN_ERR_RANGE if a V value beyond the
+ * fp16 range met the fp16 P V product, ATTN_ERR_CUDA if the synchronisation itself
+ * failed. The error word is one per device, shared by every stream and every forward
+ * launch on it (attn_fwd, attn_fwd_fp8, the host-buffer calls): it keeps the first code
+ * any of them records until a call of this function clears it, and this function waits
+ * only for `stream`. With launches on several streams, synchronise them all before
+ * reading it, or a code may be seen (and cleared) by the call for another stream.
  */
 int attn_debug_error(cudaStream_t stream, int* device_code);
 
@@ -229,8 +256,8 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* out, const
              int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
              float scale, int mask_kind, int64_t window, cudaStream_t stream);
 
-/* attn_bwd with options (wait bound and CTA count as for attn_fwd_ex; inject_stall
-   is ignored); opts may be NULL. */
+/* attn_bwd with options (wait bound and CTA count as for attn_fwd_ex; the other fields
+   are ignored); opts may be NULL. */
 int attn_bwd_ex(const void* q, const void* k, const void* v, const void* out, const float* lse,
                 const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
                 int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
@@ -289,16 +316,16 @@ int attn_bwd_debug_error(cudaStream_t stream, int* device_code);
  * synchronises. Outputs and the workspace must not overlap each other or the inputs
  * (ATTN_ERR_INVALID_ARG). A page-table entry outside [0, num_pages) that the step needs
  * is reported by attn_decode_debug_error as ATTN_ERR_INVALID_ARG (the step's result is
- * then undefined, but nothing outside the given buffers is read). Errors, bounded waits
- * and ATTN_ERR_TIMEOUT as attn_fwd.
+ * then undefined, but nothing outside the given buffers is read). Precision, the V range
+ * (ATTN_ERR_RANGE, p_bf16), errors, bounded waits and ATTN_ERR_TIMEOUT as attn_fwd.
  */
 int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
                 const int32_t* seq_lens, void* out, float* lse, void* workspace, size_t workspace_bytes,
                 int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t d,
                 int64_t num_pages, int64_t page_size, int64_t max_pages_per_seq, int64_t num_splits,
                 float scale, int mask_kind, int64_t window, cudaStream_t stream);
-/* attn_decode with options (wait bound and CTA count as for attn_fwd_ex; inject_stall
-   is ignored); opts may be NULL. */
+/* attn_decode with options (wait bound, CTA count and p_bf16 as for attn_fwd_ex;
+   inject_stall and item_visits are ignored); opts may be NULL. */
 int attn_decode_ex(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
                    const int32_t* seq_lens, void* out, float* lse, void* workspace, size_t workspace_bytes,
                    int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t d,
@@ -314,8 +341,9 @@ size_t attn_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t Nq, int64_t d,
    shorter than four tiles; -1 on invalid sizes. Host-only. */
 int64_t attn_decode_num_splits(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t max_seq_len,
                                int mask_kind, int64_t window);
-/* attn_debug_error for the decoding kernel's error word: ATTN_ERR_TIMEOUT for a wait
-   that gave up, ATTN_ERR_INVALID_ARG for a bad sequence length or page-table entry. */
+/* attn_debug_error for the decoding kernel's error word (one per device, shared like the
+   forward's): ATTN_ERR_TIMEOUT for a wait that gave up, ATTN_ERR_INVALID_ARG for a bad
+   sequence length or page-table entry, ATTN_ERR_RANGE for a V value beyond the fp16 range. */
 int attn_decode_debug_error(cudaStream_t stream, int* device_code);
 
 /*

@@ -57,6 +57,8 @@ def call(lib, q=Q, k=K, v=V, o=O, l=L, B=1, Hq=2, Hkv=2, N=256, d=64, scale=0.12
     (dict(q=Q + 8), 3), (dict(k=K + 4), 3), (dict(v=V + 2), 3), (dict(o=O + 8), 3), (dict(l=L + 2), 3),
     (dict(o=Q), 1), (dict(o=K + 64), 1), (dict(l=O + 1024), 1), (dict(l=V), 1),
     (dict(N=(1 << 30) + 1), 1),
+    # 2^60 rows x d: each factor within its bound, the byte count beyond 63 bits
+    (dict(B=1 << 10, Hq=1 << 20, Hkv=1 << 20, N=1 << 30), 1), (dict(B=1, Hq=1 << 30, Hkv=1, N=1 << 30), 1),
 ])
 def test_invalid_arguments_rejected_before_launch(lib, kw, status):
     assert call(lib, **kw) == status
@@ -113,6 +115,7 @@ def call_bwd(lib, q=Q, k=K, v=V, o=O, l=L, do=DO, dq=DQ, dk=DK, dv=DV, ws=WS, ws
 def test_backward_workspace_bytes(lib):
     assert lib.attn_bwd_workspace_bytes(2, 32, 8192) == 4 * 2 * 32 * 8192
     assert lib.attn_bwd_workspace_bytes(0, 1, 1) == 0 and lib.attn_bwd_workspace_bytes(1, 1, -1) == 0
+    assert lib.attn_bwd_workspace_bytes(1 << 30, 1 << 30, 1 << 30) == 0   # beyond 63 bits
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -124,6 +127,7 @@ def test_backward_workspace_bytes(lib):
     (dict(do=DO + 8), 3), (dict(dq=DQ + 8), 3), (dict(dk=DK + 4), 3), (dict(dv=DV + 2), 3), (dict(ws=WS + 2), 3),
     (dict(dq=Q), 1), (dict(dk=V + 64), 1), (dict(dv=DO), 1), (dict(ws=L), 1), (dict(dk=DQ + 128), 1),
     (dict(ws=DV + 256), 1),
+    (dict(B=1 << 10, Hq=1 << 20, Hkv=1 << 20, N=1 << 30), 1),
 ])
 def test_backward_invalid_arguments_rejected_before_launch(lib, kw, status):
     assert call_bwd(lib, **kw) == status
@@ -235,7 +239,9 @@ def call_merge(lib, acc=A1, accl=A2, part=P1, partl=P2, out=MO, rows=100, d=128,
 
 @pytest.mark.parametrize("kw,status", [
     (dict(acc=None), 1), (dict(accl=None), 1), (dict(part=None), 1), (dict(partl=None), 1),
-    (dict(rows=0), 1), (dict(mode=2), 1), (dict(d=96), 2),
+    (dict(rows=0), 1), (dict(mode=4), 1), (dict(mode=-1), 1), (dict(d=96), 2),
+    (dict(mode=3, part=P1 + 8), 3),                     # fp32 partials need 16-byte alignment
+    (dict(mode=3, out=P1), 1), (dict(mode=2, out=P1 + 256), 1),  # a bf16 out may not alias fp32 partials
     (dict(acc=A1 + 8), 3), (dict(part=P1 + 4), 3), (dict(out=MO + 2), 3), (dict(accl=A2 + 2), 3),
     (dict(accl=A1 + 64), 1), (dict(part=A1), 1), (dict(out=A2), 1), (dict(out=P2), 1),
 ])
@@ -250,6 +256,7 @@ def test_merge_valid_arguments_reach_the_launch(lib):
     assert call_merge(lib) == 4          # no device: the launch fails
     assert call_merge(lib, out=None, mode=0) == 4
     assert call_merge(lib, out=P1) == 4  # out may alias the partial
+    assert call_merge(lib, mode=3) == 4 and call_merge(lib, mode=2, out=None) == 4   # fp32 partials
 
 
 # ------------------------------------------------------------------ host-buffer forward
@@ -272,6 +279,7 @@ def call_host(lib, hq=HQ, hk=HK, hv=HV, ho=HO, hl=HL, q=Q, k=K, v=V, o=O, l=L, B
     (dict(o=K), 1), (dict(l=O + 64), 1),                        # device outputs overlap
     (dict(ho=HQ + 1024), 1), (dict(hl=HO + 4096), 1), (dict(hl=HV), 1),   # host outputs overlap
     (dict(fp8=True, d=64), 2), (dict(fp8=True, d=128, sq=0.0), 1), (dict(fp8=True, d=128, sv=float("nan")), 1),
+    (dict(k=V), 1), (dict(v=K), 1), (dict(k=Q + 1024), 1),       # device staging inputs overlap
 ])
 def test_host_forward_invalid_arguments_rejected_before_enqueueing(lib, kw, status):
     assert call_host(lib, **kw) == status

@@ -1,8 +1,9 @@
 """The five attention-forward workloads at full size, in the launch
 configuration the benchmark times, against the fp64 oracle on 256 seeded query
 rows per head (every row for the tiny workload): out rel-L2 <= 4e-3, lse
-max-abs <= 1e-3, out element error <= max(1e-2, one bf16 ulp of the exact
-value)."""
+max-abs <= 1e-3, out element error <= 1e-2 (above |exact| = 4, where a
+correctly rounded bf16 value alone can be 2^-6 off, only the format's extra
+rounding is added: tests.parity.element_bound)."""
 import pytest
 import torch
 
