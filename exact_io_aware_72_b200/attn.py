@@ -289,7 +289,7 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
            mask: str = "causal", window: Optional[int] = None, num_splits: Optional[int] = None,
            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
            workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
-           wait_timeout_ns: int = 0, grid_ctas: int = 0, p_bf16: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+           wait_timeout_ns: int = 0, grid_ctas: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
     """One decoding step against a paged KV cache: returns (out bf16 [B,Hq,Nq,d],
     lse fp32 [B,Hq,Nq]).
 
@@ -337,7 +337,7 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
     ws_ptr, ws_len = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    opts = FwdOptions(int(wait_timeout_ns), 0, int(grid_ctas), None, 1 if p_bf16 else 0)
+    opts = FwdOptions(int(wait_timeout_ns), 0, int(grid_ctas), None, 0, 0)
     with torch.cuda.device(q.device):
         st = lib.attn_decode_ex(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
                                 seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(), ws_ptr, ws_len,

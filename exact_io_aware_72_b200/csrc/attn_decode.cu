@@ -275,7 +275,6 @@ extern "C" int attn_decode_ex(const void* q, const void* k_cache, const void* v_
   p.num_splits = static_cast<int>(num_splits);
   p.num_items = static_cast<int>(items);
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.f16p = (opts && opts->p_bf16) ? 0 : 1;
   p.timeout_ns = (opts && opts->wait_timeout_ns) ? opts->wait_timeout_ns : kDefaultTimeoutNs;
 
   int grid = static_cast<int>(std::min<int64_t>(items, dev.sm_count));
@@ -323,8 +322,7 @@ extern "C" int attn_decode_debug_error(cudaStream_t stream, int* device_code) {
   if (cudaMemcpy(dev.err_word, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return ATTN_ERR_CUDA;
   if (device_code) *device_code = code;
   if (code == 0) return ATTN_OK;
-  if (code & (kDErrSeqLen | kDErrPage)) return ATTN_ERR_INVALID_ARG;
-  return (code & kDErrRange) ? ATTN_ERR_RANGE : ATTN_ERR_TIMEOUT;
+  return (code & (kDErrSeqLen | kDErrPage)) ? ATTN_ERR_INVALID_ARG : ATTN_ERR_TIMEOUT;
 }
 
 // ---------------------------------------------------------------- allocation-free variant

@@ -34,16 +34,15 @@
 //   ahead.  Boxes that hold no position of the step's visible range are not
 //   loaded at all; under a sliding window the pages wholly before the oldest
 //   visible key are never looked up, so a caller may recycle them (a rolling
-//   window buffer).  Before the P V MMA the softmax warps convert each V tile
-//   to fp16 in shared memory (P is fp16, 11 significant bits) and clear the
-//   rows of an edge tile outside the visible range (those slots may hold
-//   anything); masked scores are replaced by -inf.
+//   window buffer).  Rows of an edge tile outside the visible range are
+//   cleared in shared memory before the P V MMA (those slots may hold
+//   anything), and masked scores are replaced by -inf.
 //
 // CTA organisation (224 threads): warps 0-3 softmax (thread = TMEM lane),
 // warp 4 TMA loader for the work items, Q and K, warp 5 tcgen05 issuer, warp 6
 // TMA loader for V (small pages cost one TMA box each; two issuing warps keep
 // the K and V boxes of a tile going out together).  TMEM: S double buffer at columns
-// [0,128) and [128,256), P double buffer (fp16 pairs) at [256,320) and
+// [0,128) and [128,256), P double buffer (bf16 pairs) at [256,320) and
 // [320,384), O at [384, 384 + d).  All waits are bounded like the forward's.
 #pragma once
 
@@ -65,14 +64,10 @@ constexpr int kDecMmaWarp = 5;
 constexpr int kDecVLoaderWarp = 6;  // V
 constexpr uint32_t kDecTmemCols = 512;
 constexpr float kDecLn2 = 0.6931471805599453f;
-// P goes to the P V product as fp16 (11 significant bits) with V converted to
-// fp16 in shared memory, as in the forward.  A lane's running max moves only
-// when it grows by more than 2^15, so P <= 2^15 < 65504 (the largest fp16
-// value); fp32 sums and accumulators carry that, and the final merge uses the
-// same maxima.  With bf16 P (inputs whose V exceeds the fp16 range, by request)
-// the margin is 2^32, which bf16 carries.
-constexpr float kDecRescaleThreshold = 15.0f;
-constexpr float kDecRescaleThresholdBF16 = 32.0f;
+// A lane's running max moves only when it grows by more than 2^32 (as in the
+// forward): P may then exceed 1 by up to 2^32, which bf16 P and fp32 sums and
+// accumulators carry without loss, and the final merge uses the same maxima.
+constexpr float kDecRescaleThreshold = 32.0f;
 // Work items are handed out by a counter in global memory; the loader fetches
 // them and passes each index to the other roles through this many slots.
 constexpr int kItemSlots = 4;
@@ -82,7 +77,6 @@ enum : int { kDRoleLoader = 1, kDRoleMma = 2, kDRoleSoftmax = 3 };
 // Data errors recorded in the error word (bits 20..21; low bits: sequence index).
 constexpr int kDErrSeqLen = 1 << 20;   // seq_lens[b] < Nq or beyond the page table
 constexpr int kDErrPage = 2 << 20;     // a page-table entry the step needs is out of range
-constexpr int kDErrRange = 4 << 20;    // a V value fp16 cannot hold (|v| >= 2^16 or not finite), fp16 P
 
 struct DecParams {
   CUtensorMap tm_q;       // [1, B*Hq*Nq, d] bf16, box 64 x rows_chunk, 128-byte swizzle
@@ -103,7 +97,6 @@ struct DecParams {
   int mask_kind, window;
   int num_splits, num_items;
   float scale_log2;       // scale * log2(e)
-  int f16p;               // 1: P and V go to the P V product as fp16; 0: as bf16
   unsigned long long timeout_ns;
   unsigned int* sched;    // [0] next work item, [1] CTAs finished; zero between launches
 };
@@ -420,8 +413,7 @@ __device__ __forceinline__ void dec_mma(const DecParams& p, uint32_t sbase, cons
   using L = DecSmem<D>;
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
   constexpr uint32_t idesc_s = idesc_bf16_f32(kLanes, kKeys, false);
-  // fp16 P and the fp16 copy of V, or bf16 both
-  const uint32_t idesc_o = p.f16p ? idesc_f16_f32(kLanes, D, true) : idesc_bf16_f32(kLanes, D, true);
+  constexpr uint32_t idesc_o = idesc_bf16_f32(kLanes, D, true);
   const uint64_t q_desc = smem_desc_sw128(sbase + L::kQOff, 16, 1024);
   // A K tile is [half][128 rows][128 B]; a V tile is 128 / R page blocks of
   // [half][R rows][128 B] (R = rows_per_load), which for one column half or
@@ -617,7 +609,7 @@ __device__ __forceinline__ void dec_softmax(const DecParams& p, uint32_t sbase, 
       float f = 1.f;
       if (m == -INFINITY) {
         m = m_new;  // nothing accumulated yet for this lane
-      } else if (m_new > m + (p.f16p ? kDecRescaleThreshold : kDecRescaleThresholdBF16)) {
+      } else if (m_new > m + kDecRescaleThreshold) {
         f = dec_exp2(m - m_new);
         l *= f;
         m = m_new;
@@ -649,7 +641,7 @@ __device__ __forceinline__ void dec_softmax(const DecParams& p, uint32_t sbase, 
       for (int c = 0; c < C / 2; ++c) {
         const float lo = dec_exp2(x[2 * c] - mu), hi = dec_exp2(x[2 * c + 1] - mu);
         l += lo + hi;
-        pk[c] = p.f16p ? pack_f16x2(lo, hi) : dec_pack_bf16x2(lo, hi);  // round to nearest even
+        pk[c] = dec_pack_bf16x2(lo, hi);
       }
       const uint32_t p_addr = lane_addr + L::kPCol + 64 * (gi & 1) + copy * (C / 2);
       if constexpr (C == 32) {
@@ -663,63 +655,27 @@ __device__ __forceinline__ void dec_softmax(const DecParams& p, uint32_t sbase, 
           tmem_store_32cols(p_addr + c, part);
         }
       }
-      {
-        // V of this tile to fp16 in place (fp16 P), by all four softmax warps,
-        // before P is published: the P V product reads it once PFull completes.
-        // A magnitude of 2^16 or more is recorded as kDErrRange.  On an
-        // edge tile, V rows outside [lo_pos, L) were not loaded or hold slots
-        // past the sequence end; P is zero there, and they are written as zeros
-        // instead, so that 0 * (whatever they held) cannot reach O.  The tile is
-        // page blocks of R rows, each 64-column half after half (a 16-byte unit
-        // at byte o is row (o / block) * R + (o % (R * 128)) / 128, block = R *
-        // 128 * halves bytes).
+      if (base < it.lo_pos || base + kKeys > it.L) {
+        // Edge tile: V rows outside [lo_pos, L) were not loaded or hold
+        // slots past the sequence end; P is zero there, and they are cleared
+        // so that 0 * (whatever they hold) cannot reach O.
         const uint32_t vidx = 2 * gi + 1, vslot = vidx % L::kStages;
         if (!w.wait_warp(bar(L::kKVFull + vslot), (vidx / L::kStages) & 1, code | (L::kKVFull + vslot))) {
           ok = false;
           break;
         }
-        const uint32_t vbase = sbase + L::kRingOff + vslot * L::kTileBytes;
-        const bool edge = base < it.lo_pos || base + kKeys > it.L;
-        const int z0 = max(0, min(kKeys, it.lo_pos - base));  // rows [0, z0) are cleared
-        const int z1 = max(0, min(kKeys, it.L - base));       // and rows [z1, 128)
-        uint32_t mag = 0;  // per-half maximum of |v| as bf16 bits
-        if (!edge) {
-          if (p.f16p) {
-#pragma unroll 4
-            for (uint32_t e = tid; e < L::kTileBytes / 16; e += kLanes) {
-              uint32_t a, b, c2, d2;
-              ld_shared_v4(vbase + e * 16, a, b, c2, d2);
-              mag = max_u16x2(max_u16x2(mag, a & 0x7fff7fffu), max_u16x2(b & 0x7fff7fffu, c2 & 0x7fff7fffu));
-              mag = max_u16x2(mag, d2 & 0x7fff7fffu);
-              st_shared_v4(vbase + e * 16, bf16x2_to_f16x2(a), bf16x2_to_f16x2(b), bf16x2_to_f16x2(c2),
-                           bf16x2_to_f16x2(d2));
-            }
-            fence_proxy_async_smem();
-          }
-        } else {
-          // R (rows per page block) is a power of two: rows from shifts.
-          const uint32_t lg_r = static_cast<uint32_t>(__ffs(p.rows_per_load) - 1);
-          const uint32_t lg_block = lg_r + 7 + (L::kChunks == 2 ? 1 : 0);
-          const uint32_t in_block = (static_cast<uint32_t>(p.rows_per_load) << 7) - 1;
-#pragma unroll 4
-          for (uint32_t e = tid; e < L::kTileBytes / 16; e += kLanes) {
-            const uint32_t o = e * 16;
-            const int row = static_cast<int>(((o >> lg_block) << lg_r) + ((o & in_block) >> 7));
-            if (row < z0 || row >= z1) {
-              st_shared_v4(vbase + o, 0u, 0u, 0u, 0u);
-            } else if (p.f16p) {
-              uint32_t a, b, c2, d2;
-              ld_shared_v4(vbase + o, a, b, c2, d2);
-              mag = max_u16x2(max_u16x2(mag, a & 0x7fff7fffu), max_u16x2(b & 0x7fff7fffu, c2 & 0x7fff7fffu));
-              mag = max_u16x2(mag, d2 & 0x7fff7fffu);
-              st_shared_v4(vbase + o, bf16x2_to_f16x2(a), bf16x2_to_f16x2(b), bf16x2_to_f16x2(c2),
-                           bf16x2_to_f16x2(d2));
-            }
-          }
-          fence_proxy_async_smem();
+        const int z0 = max(0, min(kKeys, it.lo_pos - base));  // rows [0, z0)
+        const int z1 = max(0, min(kKeys, it.L - base));       // rows [z1, 128)
+        const int nrows = z0 + (kKeys - z1);
+        uint4* vt = reinterpret_cast<uint4*>(smem + L::kRingOff + vslot * L::kTileBytes);
+        for (int e = tid; e < nrows * 8 * L::kChunks; e += kLanes) {
+          const int rr = e / (8 * L::kChunks), rem = e - rr * (8 * L::kChunks);
+          const int row = rr < z0 ? rr : z1 + (rr - z0);
+          const int R = p.rows_per_load;
+          vt[((row / R) * R * 128 * L::kChunks + (rem >> 3) * R * 128 + (row % R) * 128) / 16 + (rem & 7)] =
+              make_uint4(0u, 0u, 0u, 0u);
         }
-        if (p.f16p && __any_sync(0xffffffffu, max(mag >> 16, mag & 0xffffu) >= 0x4780u) && (tid & 31) == 0)
-          atomicCAS(p.err, 0, kDErrRange);
+        fence_proxy_async_smem();
       }
       tmem_store_wait();
       tc_fence_before_sync();

@@ -316,16 +316,20 @@ int attn_bwd_debug_error(cudaStream_t stream, int* device_code);
  * synchronises. Outputs and the workspace must not overlap each other or the inputs
  * (ATTN_ERR_INVALID_ARG). A page-table entry outside [0, num_pages) that the step needs
  * is reported by attn_decode_debug_error as ATTN_ERR_INVALID_ARG (the step's result is
- * then undefined, but nothing outside the given buffers is read). Precision, the V range
- * (ATTN_ERR_RANGE, p_bf16), errors, bounded waits and ATTN_ERR_TIMEOUT as attn_fwd.
+ * then undefined, but nothing outside the given buffers is read). Precision: scores, sums
+ * and the split partials are fp32; P goes to the P V product rounded to bf16 (RNE), so,
+ * unlike attn_fwd, a row dominated by a few keys can be off by about one bf16 ulp of out
+ * (the step is bound by HBM reads, and an fp16 copy of V in shared memory would hold each
+ * V slot of the load ring longer, costing 15-40 % of the bandwidth). Any bf16 V is taken.
+ * Errors, bounded waits and ATTN_ERR_TIMEOUT as attn_fwd.
  */
 int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
                 const int32_t* seq_lens, void* out, float* lse, void* workspace, size_t workspace_bytes,
                 int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t d,
                 int64_t num_pages, int64_t page_size, int64_t max_pages_per_seq, int64_t num_splits,
                 float scale, int mask_kind, int64_t window, cudaStream_t stream);
-/* attn_decode with options (wait bound, CTA count and p_bf16 as for attn_fwd_ex;
-   inject_stall and item_visits are ignored); opts may be NULL. */
+/* attn_decode with options (wait bound and CTA count as for attn_fwd_ex; the other
+   fields are ignored); opts may be NULL. */
 int attn_decode_ex(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
                    const int32_t* seq_lens, void* out, float* lse, void* workspace, size_t workspace_bytes,
                    int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t d,
@@ -343,7 +347,7 @@ int64_t attn_decode_num_splits(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, i
                                int mask_kind, int64_t window);
 /* attn_debug_error for the decoding kernel's error word (one per device, shared like the
    forward's): ATTN_ERR_TIMEOUT for a wait that gave up, ATTN_ERR_INVALID_ARG for a bad
-   sequence length or page-table entry, ATTN_ERR_RANGE for a V value beyond the fp16 range. */
+   sequence length or page-table entry. */
 int attn_decode_debug_error(cudaStream_t stream, int* device_code);
 
 /*

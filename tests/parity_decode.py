@@ -7,7 +7,11 @@ import torch
 
 from harness.inputs import MASK_NAMES, make_paged_kv
 from oracle import attention_decode_fp64 as D
-from tests.parity import compare, to_np
+from tests.parity import compare, element_bound_p_bf16, to_np
+
+# Decoding rounds P to bf16 (the step is bound by HBM reads; include/attn.h):
+# its element bound is max(1e-2, one bf16 ulp of the exact value).
+DECODE_BOUND = element_bound_p_bf16
 
 
 def keep_from_for_window(lens, Nq, window):
@@ -53,7 +57,7 @@ def check_decode_case(B, Hq, Hkv, Nq, d, lens, page_size, mask, window=None, see
     out, lse = run_decode(gpu, mask, window, scale, num_splits, grid_ctas)
     ref_o, ref_l = oracle_for(inp, mask, window, scale)
     what = f"{(B, Hq, Hkv, Nq, d, tuple(int(x) for x in lens), page_size, mask, window, num_splits)}"
-    stats = compare(to_np(out), to_np(lse), ref_o, ref_l, what)
+    stats = compare(to_np(out), to_np(lse), ref_o, ref_l, what, bound=DECODE_BOUND)
     st, code = decode_debug_error()
     assert st == 0, f"{what}: device error {code:#x}"
     return stats

@@ -1,7 +1,8 @@
-"""V values beyond the fp16 range.  The default forward and decoding step feed
-P V to the tensor core in fp16; a V value of magnitude 2^16 or more is reported
-as ATTN_ERR_RANGE by the debug-error calls (the result is then undefined), and
-the bf16-P option (p_bf16) computes such inputs at its own documented bound."""
+"""V values beyond the fp16 range.  The default forward feeds P V to the tensor
+core in fp16; a V value of magnitude 2^16 or more is reported as ATTN_ERR_RANGE
+by attn_debug_error (the result is then undefined), and the bf16-P option
+(p_bf16) computes such inputs at its own documented bound.  Decoding feeds P V
+in bf16 and takes any V."""
 import numpy as np
 import pytest
 import torch
@@ -60,21 +61,16 @@ def test_forward_p_bf16_takes_any_v(cuda_ok, mask, window, d):
             extra=p_rounding_term(q, k, v, mask, window))
 
 
-def test_decode_reports_and_p_bf16_takes_any_v(cuda_ok):
+def test_decode_takes_any_v(cuda_ok):
+    # Decoding feeds P V as bf16, so any bf16 V value is taken (no range report).
     inp = make_paged_kv(2, 8, 2, 1, 128, [300, 900], 16, 44, device="cpu")
     inp["v_cache"][0, 1, 3, 7] = 2.0e5
     g = {k: t.cuda() for k, t in inp.items()}
     A.decode_debug_error()
-    run_decode(g, "causal", num_splits=2)
-    st, code = A.decode_debug_error()
-    assert st == A.ATTN_ERR_RANGE, (st, hex(code))
-    from exact_io_aware_72_b200 import decode
-    out, lse = decode(g["q"], g["k_cache"], g["v_cache"], g["block_table"], g["seq_lens"], num_splits=2,
-                      p_bf16=True)
-    torch.cuda.synchronize()
+    out, lse = run_decode(g, "causal", num_splits=2)
     assert A.decode_debug_error()[0] == 0
     ref_o, ref_l = oracle_for(inp, "causal")
-    compare(to_np(out), to_np(lse), ref_o, ref_l, "decode p_bf16", bound=element_bound_p_bf16)
+    compare(to_np(out), to_np(lse), ref_o, ref_l, "decode large v", bound=element_bound_p_bf16)
 
 
 @pytest.mark.parametrize("N", [1, 129, 1000])
