@@ -56,10 +56,12 @@ KERNEL_SOURCES = ["exact_io_aware_72_b200/csrc/attn_fwd.cu", "exact_io_aware_72_
                   "exact_io_aware_72_b200/csrc/sm100_ptx.cuh"]
 # DRAM bytes per launch of the forward kernel from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the kernel
-# sources it was taken on; reported only while the sources still match.
+# sources it was taken on; reported only while the sources still match.  The
+# long workload's figure is the capture of the same kernel on a causal
+# N = 32768 case (1, 32, 32, 32768, 128) times 4: DRAM bytes grow linearly in N.
 NCU_TRAFFIC = {
-    ("dense", "a1fe7d5cc654b746"): 407916032 + 110856192,       # profiles/attn_fwd_dense_ncu.md
-    ("dense_fp8", "a1fe7d5cc654b746"): 201595392 + 97890304,    # profiles/attn_fwd_fp8_dense_ncu.md
+    ("dense", "59529aafc8fdc7bc"): 408637696 + 110999296,
+    ("long", "59529aafc8fdc7bc"): 4 * (904199936 + 251104512),
 }
 
 
@@ -89,7 +91,7 @@ DECODE_KERNEL_SOURCES = ["exact_io_aware_72_b200/csrc/attn_decode_kernel.cuh", "
 # DRAM bytes per launch of the decoding kernel from one ncu capture, keyed by
 # workload and the hash of the decoding kernel's device sources.
 DECODE_NCU_TRAFFIC = {
-    ("decode_gqa", "32d09ba4e712aaae"): 536997632 + 3341312,   # profiles/attn_decode_gqa_ncu.md
+    ("decode_gqa", "32d09ba4e712aaae"): 536997632 + 3341312,
 }
 
 
