@@ -38,7 +38,7 @@ class FwdOptions(ctypes.Structure):
     """attn_fwd_options of include/attn.h."""
     _fields_ = [("wait_timeout_ns", ctypes.c_uint64), ("inject_stall", ctypes.c_int),
                 ("grid_ctas", ctypes.c_int), ("item_visits", ctypes.c_void_p), ("p_bf16", ctypes.c_int),
-                ("out_fp32", ctypes.c_int)]
+                ("out_fp32", ctypes.c_int), ("key_offset", ctypes.c_int64)]
 
 
 def lib_path() -> str:
@@ -116,7 +116,8 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float
         mask: str = "causal", window: Optional[int] = None, out: Optional[torch.Tensor] = None,
         lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
         wait_timeout_ns: int = 0, inject_stall: bool = False, grid_ctas: int = 0, p_bf16: bool = False,
-        item_visits: Optional[torch.Tensor] = None, out_fp32: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+        item_visits: Optional[torch.Tensor] = None, out_fp32: bool = False, key_offset: int = 0
+        ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Exact attention forward: returns (out bf16 [B,Hq,N,d], lse fp32 [B,Hq,N]).
 
     q: [B,Hq,N,d], k/v: [B,Hkv,N,d], bf16, contiguous, on one CUDA device.
@@ -125,7 +126,8 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float
     ``p_bf16`` selects bf16 P for V values beyond the fp16 range (see
     include/attn.h); ``item_visits`` (int32 CUDA tensor of num_work_items
     counters) is a test hook counting each work item's visits; ``out_fp32``
-    returns out in fp32, unrounded (partial results to merge).
+    returns out in fp32, unrounded (partial results to merge); ``key_offset``
+    places query row i at key position i + key_offset (causal and window masks).
     """
     lib = load_library()
     _check(q, "q", torch.bfloat16, 4)
@@ -154,7 +156,7 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float
             raise ValueError("item_visits must be a contiguous int32 CUDA tensor")
         visits = item_visits.data_ptr()
     opts = FwdOptions(int(wait_timeout_ns), 1 if inject_stall else 0, int(grid_ctas), visits, 1 if p_bf16 else 0,
-                      1 if out_fp32 else 0)
+                      1 if out_fp32 else 0, int(key_offset))
     with torch.cuda.device(q.device):
         st = lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                              B, Hq, Hkv, N, d, float(scale), MASKS[mask],
@@ -337,7 +339,7 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
     ws_ptr, ws_len = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    opts = FwdOptions(int(wait_timeout_ns), 0, int(grid_ctas), None, 0, 0)
+    opts = FwdOptions(int(wait_timeout_ns), 0, int(grid_ctas), None, 0, 0, 0)
     with torch.cuda.device(q.device):
         st = lib.attn_decode_ex(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
                                 seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(), ws_ptr, ws_len,

@@ -103,12 +103,13 @@ struct Plan {
 
 // Checks that need no device; fills the schedule plan.
 int check_sizes(int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d, int mask_kind, int64_t window,
-                Plan& plan) {
+                Plan& plan, int64_t key_offset = 0) {
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (mask_kind != ATTN_MASK_FULL && mask_kind != ATTN_MASK_CAUSAL && mask_kind != ATTN_MASK_SLIDING_WINDOW)
     return ATTN_ERR_INVALID_ARG;
   if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window < 1) return ATTN_ERR_INVALID_ARG;
+  if (key_offset < 0 || key_offset > (int64_t(1) << 30)) return ATTN_ERR_INVALID_ARG;
   // Index arithmetic in the kernel is 32-bit for rows and heads.
   if (N > (int64_t(1) << 30) || B * Hq > (int64_t(1) << 30) || B * Hkv > (int64_t(1) << 30))
     return ATTN_ERR_INVALID_ARG;
@@ -119,7 +120,7 @@ int check_sizes(int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d, int ma
   plan.mask_kind = mask_kind;
   plan.window = window;
   // A window covering every earlier key is plain causal attention.
-  if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window >= N) {
+  if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window >= N + key_offset) {
     plan.mask_kind = ATTN_MASK_CAUSAL;
     plan.window = N;
   }
@@ -155,7 +156,8 @@ int fwd_launch(const void* q, const void* k, const void* v, void* out, float* ls
                int64_t window, cudaStream_t stream, const attn_fwd_options* opts) {
   if (!q || !k || !v || !out || !lse) return ATTN_ERR_INVALID_ARG;
   Plan plan{};
-  int st = check_sizes(B, Hq, Hkv, N, d, mask_kind, window, plan);
+  const int64_t key_offset = opts ? opts->key_offset : 0;
+  int st = check_sizes(B, Hq, Hkv, N, d, mask_kind, window, plan, key_offset);
   if (st != ATTN_OK) return st;
   if (eb == 1 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (!std::isfinite(score_scale) || !(score_scale > 0.f) || !std::isfinite(v_scale) || !(v_scale > 0.f))
@@ -197,7 +199,8 @@ int fwd_launch(const void* q, const void* k, const void* v, void* out, float* ls
   p.N = static_cast<int>(N);
   p.group = static_cast<int>(Hq / Hkv);
   p.mask_kind = plan.mask_kind;
-  p.window = static_cast<int>(plan.mask_kind == ATTN_MASK_SLIDING_WINDOW ? plan.window : N);
+  p.window = static_cast<int>(plan.mask_kind == ATTN_MASK_SLIDING_WINDOW ? std::min<int64_t>(plan.window, 1 << 30) : N);
+  p.key_offset = plan.mask_kind == ATTN_MASK_FULL ? 0 : static_cast<int>(key_offset);
   p.scale_log2 = score_scale * 1.4426950408889634f;
   p.v_scale = v_scale;
   p.pair_heads = plan.pair_heads;

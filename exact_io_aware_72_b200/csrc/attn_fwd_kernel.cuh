@@ -106,6 +106,7 @@ struct FwdParams {
   int group;         // Hq / Hkv
   int mask_kind;
   int window;
+  int key_offset;    // query row i sits at key position i + key_offset (causal and window masks)
   float scale_log2;  // scale * log2(e)
   int pair_heads;    // 1: the two tiles are two heads of one KV group
   int num_mblk;      // ceil(N / 128)
@@ -161,6 +162,11 @@ struct WorkItem {
   int lo_u, hi_u;    // union of the two ranges
 };
 
+// Row r sees keys [r + key_offset - window + 1, r + key_offset] (window), keys
+// [0, r + key_offset] (causal), or every key (full), within [0, N).  A query
+// block whose rows see no key at all (possible only with a key offset) gets one
+// tile, fully masked: its rows then end with O = 0 and lse = -inf, and no work
+// item is ever empty.
 __device__ __forceinline__ void kv_range(const FwdParams& p, int m, int& lo, int& hi) {
   const int r0 = m * kBlockM;
   const int r1 = min(r0 + kBlockM - 1, p.N - 1);
@@ -168,8 +174,8 @@ __device__ __forceinline__ void kv_range(const FwdParams& p, int m, int& lo, int
     lo = 0;
     hi = p.num_mblk - 1;
   } else {
-    hi = r1 / kBlockN;
-    lo = (p.mask_kind == kMaskWindow) ? max(0, r0 - p.window + 1) / kBlockN : 0;
+    hi = min(r1 + p.key_offset, p.N - 1) / kBlockN;
+    lo = (p.mask_kind == kMaskWindow) ? min(max(0, r0 + p.key_offset - p.window + 1) / kBlockN, hi) : 0;
   }
 }
 
@@ -211,7 +217,7 @@ __device__ __forceinline__ WorkItem decode_item(const FwdParams& p, int hu, int 
 
 // Does KV tile j need element-wise masking for query block m?
 __device__ __forceinline__ bool tile_is_partial(const FwdParams& p, int m, int j) {
-  const int r0 = m * kBlockM, c0 = j * kBlockN;
+  const int r0 = m * kBlockM + p.key_offset, c0 = j * kBlockN;
   bool partial = (c0 + kBlockN > p.N);
   if (p.mask_kind != kMaskFull) partial |= (c0 + kBlockN - 1 > r0);
   if (p.mask_kind == kMaskWindow) partial |= (c0 <= r0 + kBlockM - 1 - p.window);
@@ -709,8 +715,8 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t sbase,
         for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
         if (tile_is_partial(p, mblk, j)) {
           const int c0 = j * kBlockN;
-          const int hi_i = ((p.mask_kind == kMaskFull) ? p.N - 1 : min(row, p.N - 1)) - c0;
-          const int lo_i = (p.mask_kind == kMaskWindow) ? row - p.window + 1 - c0 : -1;
+          const int hi_i = ((p.mask_kind == kMaskFull) ? p.N - 1 : min(row + p.key_offset, p.N - 1)) - c0;
+          const int lo_i = (p.mask_kind == kMaskWindow) ? row + p.key_offset - p.window + 1 - c0 : -1;
 #pragma unroll
           for (int i = 0; i < 128; ++i)
             if (i > hi_i || i < lo_i) s[i] = -INFINITY;

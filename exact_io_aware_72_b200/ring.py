@@ -14,9 +14,14 @@ from rank r-1 (NCCL send/recv into local buffers, overlapped with the work).
 For each (query half i, key half j) block the sm_100a forward kernel computes
 a partial result with the block's own mask -- causal: every key of half j < i
 is visible ("full"), j == i is the causal diagonal, j > i is skipped; full:
-every block -- written in fp32, and ``attn_merge`` folds it into an fp32
-accumulator by its log-sum-exp; only the final merged rows are rounded to
-bf16.  The merged rows equal the exact attention of the whole sequence.
+every block; sliding window w: the block of key half j < i is a window whose
+queries sit (i - j) * h positions after its keys (the forward's ``key_offset``),
+skipped when no row reaches back into it -- written in fp32, and
+``attn_merge`` folds it into an fp32 accumulator by its log-sum-exp; only the
+final merged rows are rounded to bf16.  The merged rows equal the exact
+attention of the whole sequence ("Efficient attention: long context and
+sub-quadratic variants", stanleyjacob.dev, section "Sliding-window and local
+attention", for the window: query i sees keys i - w < j <= i).
 
 Only the data movement and the loop live here; every arithmetic step runs in
 the library's CUDA kernels (``fwd`` and ``merge``).  ``local_attention`` and
@@ -59,7 +64,7 @@ def block_mask(qi: int, kj: int, mask: str) -> Optional[str]:
     if mask == "full":
         return "full"
     if mask != "causal":
-        raise ValueError("ring attention supports the full and causal masks")
+        raise ValueError("block_mask takes the full and causal masks (block_plan also windows)")
     if kj < qi:
         return "full"
     if kj == qi:
@@ -67,10 +72,28 @@ def block_mask(qi: int, kj: int, mask: str) -> Optional[str]:
     return None
 
 
-def _default_local(q, k, v, mask, scale):
+def block_plan(qi: int, kj: int, mask: str, window: Optional[int] = None, half: Optional[int] = None
+               ) -> Optional[Tuple[str, int]]:
+    """(mask, key offset) of the (query half qi, key half kj) block, or None when no
+    key of it is visible.  Halves hold ``half`` positions; with a sliding window the
+    block's query row r sits at key position r + (qi - kj) * half."""
+    if mask != "sliding_window":
+        m = block_mask(qi, kj, mask)
+        return None if m is None else (m, 0)
+    if window is None or window < 1 or half is None or half < 1:
+        raise ValueError("a sliding window needs window >= 1 and the half length")
+    if kj > qi:
+        return None
+    offset = (qi - kj) * half
+    if offset > half + window - 2:        # even row 0's window starts after the block's last key
+        return None
+    return "sliding_window", offset
+
+
+def _default_local(q, k, v, mask, scale, window=None, key_offset=0):
     # Block results stay fp32 (unrounded) until the last merge rounds out to bf16 once.
     from .attn import fwd
-    return fwd(q, k, v, scale=scale, mask=mask, out_fp32=True)
+    return fwd(q, k, v, scale=scale, mask=mask, window=window, key_offset=key_offset, out_fp32=True)
 
 
 def _default_merge(acc_o, acc_l, part_o, part_l, first, out):
@@ -81,21 +104,22 @@ def _default_merge(acc_o, acc_l, part_o, part_l, first, out):
 def rank_forward(rank: int, world: int, q_halves: Sequence[torch.Tensor],
                  kv_at_step: Callable[[int], Tuple[Sequence[torch.Tensor], Sequence[torch.Tensor]]],
                  mask: str = "causal", scale: Optional[float] = None,
-                 local_attention: Callable = _default_local, merge: Callable = _default_merge
-                 ) -> Tuple[List[torch.Tensor], List[torch.Tensor]]:
+                 local_attention: Callable = _default_local, merge: Callable = _default_merge,
+                 window: Optional[int] = None) -> Tuple[List[torch.Tensor], List[torch.Tensor]]:
     """One rank's share of ring attention.  ``kv_at_step(s)`` returns the K and V
     halves of rank (rank - s) mod world (waiting for them to arrive if needed).
     Returns ([out_a, out_b] bf16, [lse_a, lse_b] fp32) for the rank's two query halves."""
     qids = half_ids(world, rank)
+    half = q_halves[0].shape[-2]
     # Which blocks each query half takes, in step order, so the last one can also write bf16 out.
     plan = [[] for _ in range(2)]
     for s in range(world):
         kids = half_ids(world, (rank - s) % world)
         for a in range(2):
             for b in range(2):
-                m = block_mask(qids[a], kids[b], mask)
-                if m is not None:
-                    plan[a].append((s, b, m))
+                bp = block_plan(qids[a], kids[b], mask, window, half)
+                if bp is not None:
+                    plan[a].append((s, b) + bp)
     # The accumulator is fp32 (or the inputs' dtype when that is wider); out has the inputs' dtype.
     acc_t = torch.float32 if q_halves[0].element_size() < 4 else q_halves[0].dtype
     acc_o = [torch.empty(q.shape, dtype=acc_t, device=q.device) for q in q_halves]
@@ -105,10 +129,14 @@ def rank_forward(rank: int, world: int, q_halves: Sequence[torch.Tensor],
     for s in range(world):
         k_h, v_h = kv_at_step(s)
         for a in range(2):
-            for (step, b, m) in plan[a]:
+            for (step, b, m, offset) in plan[a]:
                 if step != s:
                     continue
-                o, lse = local_attention(q_halves[a], k_h[b], v_h[b], m, scale)
+                if m == "sliding_window":
+                    o, lse = local_attention(q_halves[a], k_h[b], v_h[b], m, scale, window=window,
+                                             key_offset=offset)
+                else:
+                    o, lse = local_attention(q_halves[a], k_h[b], v_h[b], m, scale)
                 last = done[a] == len(plan[a]) - 1
                 merge(acc_o[a], acc_l[a], o, lse, done[a] == 0, outs[a] if last else None)
                 done[a] += 1
@@ -117,7 +145,8 @@ def rank_forward(rank: int, world: int, q_halves: Sequence[torch.Tensor],
 
 def ring_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask: str = "causal",
                  scale: Optional[float] = None, group=None, local_attention: Callable = _default_local,
-                 merge: Callable = _default_merge) -> Tuple[List[torch.Tensor], List[torch.Tensor]]:
+                 merge: Callable = _default_merge, window: Optional[int] = None
+                 ) -> Tuple[List[torch.Tensor], List[torch.Tensor]]:
     """Ring attention across the ranks of ``group`` (torch.distributed, NCCL for
     CUDA tensors).  q, k, v are this rank's zigzag halves stacked on a leading
     axis of 2: q [2, B, Hq, h, d], k and v [2, B, Hkv, h, d] (see
@@ -147,7 +176,7 @@ def ring_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask: str = 
             pending = dist.batch_isend_irecv(ops)
         return (cur[0][0], cur[0][1]), (cur[1][0], cur[1][1])
 
-    outs, lses = rank_forward(rank, world, (q[0], q[1]), kv_at_step, mask, scale, local_attention, merge)
+    outs, lses = rank_forward(rank, world, (q[0], q[1]), kv_at_step, mask, scale, local_attention, merge, window)
     for r in pending:
         r.wait()
     return outs, lses
@@ -160,7 +189,8 @@ def emulate_shares(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, world: int
 
 
 def run_emulated(shares, mask: str = "causal", scale: Optional[float] = None,
-                 local_attention: Callable = _default_local, merge: Callable = _default_merge):
+                 local_attention: Callable = _default_local, merge: Callable = _default_merge,
+                 window: Optional[int] = None):
     """All ranks of the ring one after the other in this process (the K/V halves a
     rank would receive are taken from the other ranks' shares directly).
     Returns every rank's ((out_a, out_b), (lse_a, lse_b))."""
@@ -170,15 +200,16 @@ def run_emulated(shares, mask: str = "causal", scale: Optional[float] = None,
         def kv_at_step(s, r=r):
             src = (r - s) % world
             return shares[src][1], shares[src][2]
-        o, l = rank_forward(r, world, shares[r][0], kv_at_step, mask, scale, local_attention, merge)
+        o, l = rank_forward(r, world, shares[r][0], kv_at_step, mask, scale, local_attention, merge, window)
         results.append(((o[0], o[1]), (l[0], l[1])))
     return results
 
 
 def ring_forward_emulated(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, world: int, mask: str = "causal",
                           scale: Optional[float] = None, local_attention: Callable = _default_local,
-                          merge: Callable = _default_merge) -> Tuple[torch.Tensor, torch.Tensor]:
+                          merge: Callable = _default_merge, window: Optional[int] = None
+                          ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Ring attention of ``world`` ranks emulated in this process on full [B, H, N, d]
     tensors; returns the reassembled (out, lse)."""
-    res = run_emulated(emulate_shares(q, k, v, world), mask, scale, local_attention, merge)
+    res = run_emulated(emulate_shares(q, k, v, world), mask, scale, local_attention, merge, window)
     return zigzag_gather([r[0] for r in res]), zigzag_gather([r[1] for r in res])

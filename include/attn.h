@@ -107,6 +107,11 @@ typedef struct {
   int out_fp32;             /* forward: 1 = out is fp32 [B, Hq, N, d] (16-byte aligned) and
                                receives O / l unrounded, for partial results that are merged
                                afterwards (attn_merge mode 2 or 3); 0 = bf16 out */
+  int64_t key_offset;       /* forward, causal and window masks: query row i sits at key
+                               position i + key_offset (>= 0), so it sees keys j <= i + key_offset
+                               (and, with a window, j > i + key_offset - window), e.g. a query
+                               block against an earlier key block in ring attention; rows that
+                               see no key end with out 0 and lse -inf. 0 = the square masks */
 } attn_fwd_options;
 
 /* attn_fwd with options (same arguments, same checks); opts may be NULL. */

@@ -144,3 +144,41 @@ def test_emulated_ring_replays_from_a_cuda_graph(cuda_ok):
         for (eo, el), (co, cl) in zip(eager, captured):
             for a, b in zip(eo + el, co + cl):
                 assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("world,window", [(2, 1), (2, 300), (2, 512), (4, 100), (4, 256), (4, 700), (8, 129),
+                                          (8, 1000), (4, 2048)])
+def test_emulated_ring_with_a_window_matches_oracle(cuda_ok, world, window):
+    # Blocks against earlier key halves are windows with a key offset (the forward's
+    # key_offset); blocks no row reaches are skipped.  Whole sequence against the oracle.
+    q, k, v = make_qkv(1, 4, 2, 2048, 128, world + window)
+    out, lse = ring.ring_forward_emulated(q.cuda(), k.cuda(), v.cuda(), world, "sliding_window", window=window)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.attention(to_np(q), to_np(k), to_np(v), None, 2, window)
+    compare(to_np(out), to_np(lse), ref_o, ref_l, f"ring world {world} window {window}")
+
+
+def test_key_offset_identities(cuda_ok):
+    from exact_io_aware_72_b200 import fwd
+    q, k, v = (t.cuda() for t in make_qkv(1, 4, 2, 700, 128, 77))
+    for mask, window in (("causal", None), ("sliding_window", 150)):
+        a = fwd(q, k, v, mask=mask, window=window)
+        b = fwd(q, k, v, mask=mask, window=window, key_offset=0)
+        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    # every key is at or before every query: causal equals full
+    full = fwd(q, k, v, mask="full")
+    for off in (700, 701, 5000):
+        c = fwd(q, k, v, mask="causal", key_offset=off)
+        assert torch.equal(c[0], full[0]) and torch.equal(c[1], full[1])
+    # a window that reaches the whole block from every row is full too
+    c = fwd(q, k, v, mask="sliding_window", window=1400, key_offset=700)
+    assert torch.equal(c[0], full[0]) and torch.equal(c[1], full[1])
+    # rows whose window starts after the last key see nothing: out 0, lse -inf
+    off, w = 900, 400
+    o, l = fwd(q, k, v, mask="sliding_window", window=w, key_offset=off)
+    torch.cuda.synchronize()
+    rows = torch.arange(700, device="cuda")
+    empty = rows + off - w + 1 > 699
+    assert empty.any() and (~empty).any()
+    assert torch.all(o[:, :, empty] == 0) and torch.all(torch.isneginf(l[:, :, empty]))
+    assert torch.isfinite(l[:, :, ~empty]).all()
