@@ -573,7 +573,10 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sbase, uin
       if (!wait_all(bar(L::kPFull + t), p_cnt & 1, code | (L::kPFull + t))) return false;
       ++p_cnt;
       const uint32_t vslot = vn % L::kStages;
-      if (!wait_all(bar(L::kKVFull + vslot), (vn / L::kStages) & 1, code | (L::kKVFull + vslot))) return false;
+      // With fp16 P the conversion barrier below implies the tile landed (its
+      // converters waited for that), and the product reads only bytes they rewrote.
+      if (!kConvV && !wait_all(bar(L::kKVFull + vslot), (vn / L::kStages) & 1, code | (L::kKVFull + vslot)))
+        return false;
       if constexpr (kConvV) {
         // Warp 11 and both MMA warps have converted this V tile (K/V step vn / 2) to fp16.
         const uint32_t v = vn >> 1;
