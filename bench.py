@@ -478,22 +478,28 @@ def bwd_cpu_baseline(w, q, k, v, do, target_s=15.0):
 
 
 def run_backward(args, w):
-    """Backward pass on one GPU: each step is one attn_bwd call (D, dQ and
-    dK/dV kernels) on the forward's out and lse and a seeded dO."""
+    """Backward pass on one GPU: each step is one attn_bwd call on the forward's
+    out and lse and a seeded dO (three kernels: D, then for d = 128 the fused
+    key-tile kernel and the dQ conversion after zeroing the fp32 dQ sums, for
+    d = 64 the dQ and dK/dV kernels)."""
     from harness.inputs import make_dout
     from exact_io_aware_72_b200 import bwd, fwd
+    from exact_io_aware_72_b200.attn import load_library
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, device=device, sharp=w.sharp)
     do = make_dout(w.B, w.Hq, w.N, w.d, w.seed, device=device)
     out, lse = fwd(q, k, v, scale=w.scale, mask=w.mask, window=w.window)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(w.B * w.Hq * w.N, dtype=torch.float32, device=device)
+    det = bool(args.bwd_deterministic)
+    fused = w.d == 128 and not det
+    ws_bytes = int(load_library().attn_bwd_workspace_bytes(w.B, w.Hq, w.N)) if fused else 4 * w.B * w.Hq * w.N
+    ws = torch.empty(ws_bytes // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
 
     def step():
         bwd(q, k, v, out, lse, do, scale=w.scale, mask=w.mask, window=w.window, dq=dq, dk=dk, dv=dv,
-            workspace=ws, stream=stream)
+            workspace=ws, stream=stream, deterministic=det)
 
     clocks = ClockSampler(0)
     clocks.start()
@@ -522,7 +528,8 @@ def run_backward(args, w):
         "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "mask": w.mask,
-                   "window": w.window, "sharp_rows": w.sharp, "l2": "inputs larger than L2 (no flush)"},
+                   "window": w.window, "sharp_rows": w.sharp, "l2": "inputs larger than L2 (no flush)",
+                   "bwd_path": "fused key-tile kernel" if fused else "dQ kernel + dK/dV kernel"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "traffic": None, "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak))},
@@ -762,6 +769,8 @@ def main():
                     help="B,Hq,Hkv,N,d: run this shape instead of a named workload (profiling sweeps)")
     ap.add_argument("--mask", choices=["full", "causal", "sliding_window"], default=None)
     ap.add_argument("--window", type=int, default=None)
+    ap.add_argument("--bwd-deterministic", action="store_true",
+                    help="--pass bwd with d = 128: the two-kernel path (dq bitwise reproducible)")
     ap.add_argument("--pass", dest="which", choices=["fwd", "bwd", "decode", "ring"], default="fwd",
                     help="bwd: the backward pass; decode: a paged-KV decoding step; ring: ring attention with "
                          "its ranks emulated on one GPU (one GPU each)")

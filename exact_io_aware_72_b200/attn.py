@@ -38,7 +38,7 @@ class FwdOptions(ctypes.Structure):
     """attn_fwd_options of include/attn.h."""
     _fields_ = [("wait_timeout_ns", ctypes.c_uint64), ("inject_stall", ctypes.c_int),
                 ("grid_ctas", ctypes.c_int), ("item_visits", ctypes.c_void_p), ("p_bf16", ctypes.c_int),
-                ("out_fp32", ctypes.c_int), ("key_offset", ctypes.c_int64)]
+                ("out_fp32", ctypes.c_int), ("key_offset", ctypes.c_int64), ("bwd_deterministic", ctypes.c_int)]
 
 
 def lib_path() -> str:
@@ -215,13 +215,17 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, ls
         dout: torch.Tensor, scale: Optional[float] = None, mask: str = "causal", window: Optional[int] = None,
         dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
         workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
-        wait_timeout_ns: int = 0, grid_ctas: int = 0) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+        wait_timeout_ns: int = 0, grid_ctas: int = 0,
+        deterministic: bool = False) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Exact attention backward: returns (dq, dk, dv), the gradients of
     sum(dout * out) for the forward's q, k, v (same scale / mask / window).
 
     ``out`` and ``lse`` are the forward's outputs for these inputs. The fp32
-    workspace (B*Hq*N floats, allocated here when not given) holds the row
-    terms D = rowsum(dout * out) between the kernels of this call.
+    workspace (allocated here when not given) holds the row terms
+    D = rowsum(dout * out) and, for d = 128, the fp32 sums of dq: B*Hq*N floats
+    for d = 64 or ``deterministic``, ``attn_bwd_workspace_bytes(B, Hq, N)`` bytes
+    for d = 128.  ``deterministic`` runs d = 128 on the two-kernel path (dq bitwise
+    reproducible; seven matmuls per pair instead of five).
     """
     lib = load_library()
     for t, name in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
@@ -243,7 +247,8 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, ls
         _check(t, name, torch.bfloat16, 4)
         if t.shape != ref.shape:
             raise ValueError(f"{name} has the wrong shape")
-    ws_bytes = int(lib.attn_bwd_workspace_bytes(B, Hq, N))
+    fused = d == 128 and not deterministic
+    ws_bytes = int(lib.attn_bwd_workspace_bytes(B, Hq, N)) if fused else 4 * B * Hq * N
     if workspace is None:
         workspace = torch.empty(ws_bytes // 4, dtype=torch.float32, device=q.device)
     if not (workspace.is_cuda and workspace.is_contiguous()):
@@ -251,6 +256,7 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, ls
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     opts = FwdOptions(int(wait_timeout_ns), 0, int(grid_ctas))
+    opts.bwd_deterministic = int(bool(deterministic))
     with torch.cuda.device(q.device):
         st = lib.attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                              dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),

@@ -1,6 +1,8 @@
 // Host side of the backward entry points declared in include/attn.h: argument
-// checks, TMA tensor maps and the three launches (D, dQ, dK/dV) on the
-// caller's stream.
+// checks, TMA tensor maps and the launches on the caller's stream: D, then for
+// d = 128 the zeroed fp32 dQ accumulator, the fused key-tile kernel and the dQ
+// conversion; for d = 64 (or d = 128 with bwd_deterministic) the query-tile (dQ)
+// and key-tile (dK, dV) kernels.
 #include "attn.h"
 
 #include <cuda.h>
@@ -78,7 +80,8 @@ int bwd_device_setup(BwdDevice& out) {
       if (cudaGetSymbolAddress(&addr, g_attn_bwd_error) != cudaSuccess) return ATTN_ERR_CUDA;
       info.err_word = static_cast<int*>(addr);
       if (set_smem<64, kBKernelDq>() != cudaSuccess || set_smem<64, kBKernelDkdv>() != cudaSuccess ||
-          set_smem<128, kBKernelDq>() != cudaSuccess || set_smem<128, kBKernelDkdv>() != cudaSuccess)
+          set_smem<128, kBKernelDq>() != cudaSuccess || set_smem<128, kBKernelDkdv>() != cudaSuccess ||
+          set_smem<128, kBKernelFused>() != cudaSuccess)
         return ATTN_ERR_CUDA;
     }
     info.probed = true;
@@ -111,7 +114,7 @@ template <int D, int KIND>
 cudaError_t launch_bwd(const BwdParams& p, int grid, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kBwdThreads);
+  cfg.blockDim = dim3(bwd_threads<KIND>());
   cfg.dynamicSmemBytes = BwdSmem<D>::kAlloc;
   cfg.stream = stream;
   return cudaLaunchKernelEx(&cfg, attn_bwd_kernel<D, KIND>, p);
@@ -119,13 +122,25 @@ cudaError_t launch_bwd(const BwdParams& p, int grid, cudaStream_t stream) {
 
 }  // namespace
 
+namespace {
+// Workspace of a backward: D (B*Hq*N floats), then for the fused path
+// (acc_d = 128), from the next 256-byte boundary, the fp32 dQ accumulator
+// (B*Hq*N*acc_d floats).  0 when the byte count would not fit in 62 bits.
+size_t bwd_workspace_bytes(int64_t B, int64_t Hq, int64_t N, int64_t acc_d) {
+  if (B < 1 || Hq < 1 || N < 1 || B > (int64_t(1) << 30) || Hq > (int64_t(1) << 30) || N > (int64_t(1) << 30) ||
+      B * Hq > (int64_t(1) << 61) / (N * 4 * (1 + 128)))
+    return 0;
+  const size_t rows = static_cast<size_t>(B) * static_cast<size_t>(Hq) * static_cast<size_t>(N);
+  const size_t delta = rows * sizeof(float);
+  if (acc_d == 0) return delta;
+  return ((delta + 255) & ~size_t(255)) + rows * static_cast<size_t>(acc_d) * sizeof(float);
+}
+}  // namespace
+
 extern "C" {
 
 size_t attn_bwd_workspace_bytes(int64_t B, int64_t Hq, int64_t N) {
-  if (B < 1 || Hq < 1 || N < 1 || B > (int64_t(1) << 30) || Hq > (int64_t(1) << 30) || N > (int64_t(1) << 30) ||
-      B * Hq > (int64_t(1) << 61) / (N * 4))
-    return 0;
-  return static_cast<size_t>(B) * static_cast<size_t>(Hq) * static_cast<size_t>(N) * sizeof(float);
+  return bwd_workspace_bytes(B, Hq, N, 128);  // covers every supported head dimension
 }
 
 int attn_bwd_ex(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
@@ -141,8 +156,9 @@ int attn_bwd_ex(const void* q, const void* k, const void* v, const void* out, co
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   // Byte counts must fit in 63 bits (B * Hq * N <= 2^60 after sizes_ok).
   if (B * Hq * N > (int64_t(1) << 61) / (d * 4)) return ATTN_ERR_INVALID_ARG;
-  const size_t ws = attn_bwd_workspace_bytes(B, Hq, N);
-  if (workspace_bytes < ws) return ATTN_ERR_INVALID_ARG;
+  const bool fused = (d == 128) && !(opts && opts->bwd_deterministic);
+  const size_t ws = bwd_workspace_bytes(B, Hq, N, fused ? 128 : 0);
+  if (ws == 0 || workspace_bytes < ws) return ATTN_ERR_INVALID_ARG;
   const size_t q_bytes = static_cast<size_t>(B * Hq * N * d) * 2;
   const size_t kv_bytes = static_cast<size_t>(B * Hkv * N * d) * 2;
   const size_t lse_bytes = static_cast<size_t>(B * Hq * N) * 4;
@@ -158,7 +174,8 @@ int attn_bwd_ex(const void* q, const void* k, const void* v, const void* out, co
   }
   auto mis16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
   if (mis16(q) || mis16(k) || mis16(v) || mis16(out) || mis16(dout) || mis16(dq) || mis16(dk) || mis16(dv) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 || (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(workspace) & (fused ? 15u : 3u)) != 0)
     return ATTN_ERR_MISALIGNED;
 
   BwdDevice info;
@@ -212,6 +229,21 @@ int attn_bwd_ex(const void* q, const void* k, const void* v, const void* out, co
   int sms = info.sm_count;
   if (opts && opts->grid_ctas > 0) sms = opts->grid_ctas;
   cudaError_t e;
+  if (fused) {
+    // Fused: dK, dV and the fp32 dQ sums in one key-tile kernel, then dQ to bf16.
+    const size_t acc_off = (static_cast<size_t>(rows) * sizeof(float) + 255) & ~size_t(255);
+    float* acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + acc_off);
+    const size_t acc_bytes = static_cast<size_t>(rows) * 128 * sizeof(float);
+    if (cudaMemsetAsync(acc, 0, acc_bytes, stream) != cudaSuccess) return ATTN_ERR_CUDA;
+    p.dq_acc = acc;
+    p.num_items = static_cast<int>(B * Hkv * p.num_blk);  // one key tile per item
+    const int grid = static_cast<int>(std::min<int64_t>(sms, p.num_items));
+    if (launch_bwd<128, kBKernelFused>(p, grid, stream) != cudaSuccess) return ATTN_ERR_CUDA;
+    const int64_t groups8 = rows * 128 / 8;
+    const unsigned cblocks = static_cast<unsigned>(std::min<int64_t>((groups8 + 255) / 256, int64_t(info.sm_count) * 16));
+    attn_bwd_dq_convert_kernel<<<cblocks, 256, 0, stream>>>(acc, static_cast<__nv_bfloat16*>(dq), scale, groups8);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
   p.num_items = static_cast<int>(B * Hq * p.num_blk);  // dQ: one query tile per item
   int grid = static_cast<int>(std::min<int64_t>(sms, p.num_items));
   e = (d == 128) ? launch_bwd<128, kBKernelDq>(p, grid, stream) : launch_bwd<64, kBKernelDq>(p, grid, stream);

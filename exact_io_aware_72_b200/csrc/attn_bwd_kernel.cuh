@@ -10,22 +10,30 @@
 //   dQ = scale dS K,  dK = scale dS^T Q,
 // and grouped KV heads sum the gradients of the query heads that read them.
 //
-// Three kernels, all on the caller's stream:
+// Kernels, all on the caller's stream:
 //   attn_bwd_delta_kernel  D = rowsum(dO * O) in fp32 (the caller's workspace)
-//   attn_bwd_dq_kernel     one 128-row query tile per work item, walking its
-//                          visible K/V tiles: S = Q K^T and dP = dO V^T on the
-//                          tensor core, dS by the softmax warps, dQ += dS K
-//   attn_bwd_dkdv_kernel   one 128-key K/V tile per work item, walking the
+//   the key-tile kernel    one 128-key K/V tile per work item, walking the
 //                          visible query tiles of every query head of its KV
 //                          group: S^T = K Q^T, dP^T = V dO^T, P^T and dS^T by
-//                          the softmax warps, dV += P^T dO, dK += dS^T Q
-// so every accumulator stays in TMEM for a whole work item and nothing is
-// accumulated through global atomics.
+//                          the elementwise warps, dV += P^T dO, dK += dS^T Q
+//                          (accumulated in TMEM over the item)
+// and, for dQ, one of two designs:
+//   d = 128: the key-tile kernel also forms dQ^T = K^T dS^T for each 64-query
+//            half (dS^T staged in shared memory), four more warps read it from
+//            TMEM and add it into an fp32 dQ accumulator in the workspace with
+//            coalesced global reductions, and attn_bwd_dq_convert_kernel
+//            scales and rounds the sums to bf16.  P and dS are formed once
+//            per (query, key) pair: five matmuls per pair.
+//   d = 64:  a query-tile kernel (one 128-row query tile per work item,
+//            walking its visible K/V tiles: S = Q K^T and dP = dO V^T
+//            recomputed, dS by the elementwise warps, dQ += dS K in TMEM),
+//            seven matmuls per pair and no atomics.
 //
-// CTA organisation of both tcgen05 kernels (192 threads, one CTA per SM,
-// persistent): warps 0-3 elementwise (thread = TMEM lane = one row of the
-// work item's tile), warp 4 TMA loader, warp 5 tcgen05 issuer (one elected
-// lane issues).  All waits are bounded like the forward's.
+// CTA organisation of the tcgen05 kernels (one CTA per SM, persistent):
+// warps 0-3 elementwise (thread = TMEM lane = one row of the work item's
+// tile), warp 4 TMA loader, warp 5 tcgen05 issuer (one elected lane
+// issues), and in the fused d = 128 kernel warps 6-9 reading dQ^T out of
+// TMEM.  All waits are bounded like the forward's.
 #pragma once
 
 #include <cuda.h>
@@ -40,13 +48,16 @@ using namespace attn_sm100;
 constexpr int kTile = 128;  // rows of every Q / dO / K / V tile
 constexpr int kHalf = 64;   // keys (dQ kernel) or queries (dK/dV kernel) per score half
 constexpr int kBwdThreads = 192;
+constexpr int kBwdThreadsFused = 320;
 constexpr int kBwdLoaderWarp = 4;
 constexpr int kBwdMmaWarp = 5;
+constexpr int kBwdDqWarp0 = 6;  // fused kernel: warps 6-9 read dQ^T
 constexpr uint32_t kBwdTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int { kBMaskFull = 0, kBMaskCausal = 1, kBMaskWindow = 2 };
-enum : int { kBRoleLoader = 1, kBRoleMma = 2, kBRoleElem = 3, kBKernelDq = 0, kBKernelDkdv = 1 };
+enum : int { kBRoleLoader = 1, kBRoleMma = 2, kBRoleElem = 3, kBRoleDq = 4 };
+enum : int { kBKernelDq = 0, kBKernelDkdv = 1, kBKernelFused = 2 };
 
 struct BwdParams {
   CUtensorMap tm_q;   // [B*Hq, N, d] bf16, box 64 x 128, 128-byte swizzle
@@ -58,6 +69,7 @@ struct BwdParams {
   __nv_bfloat16* dq;  // [B*Hq, N, d]
   __nv_bfloat16* dk;  // [B*Hkv, N, d]
   __nv_bfloat16* dv;  // [B*Hkv, N, d]
+  float* dq_acc;      // fused kernel: [B*Hq, N, d] fp32 dQ / scale, zeroed before the launch
   int* err;           // device error word (shared with the forward)
   int B, Hq, Hkv, N, group;
   int mask_kind, window;
@@ -157,6 +169,13 @@ __device__ __forceinline__ void tmem_load_2x32cols(uint32_t ta, uint32_t tb, uin
       : "memory");
 }
 
+// 4-byte asynchronous copy global -> shared; with src_bytes = 0 it writes zero.
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ float bexp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -208,8 +227,13 @@ struct BwdSmem {
   static constexpr int kStages = (D == 128) ? 2 : 4;
   static constexpr uint32_t kFixOff = 0;                        // two fixed tiles
   static constexpr uint32_t kRingOff = 2 * kTileBytes;          // stages of two tiles
-  static constexpr uint32_t kVecOff = kRingOff + kStages * 2 * kTileBytes;  // 4 warps x (lse2, D) x 128 floats
-  static constexpr uint32_t kBarOff = kVecOff + 4 * 2 * kTile * 4;
+  // Per-step query vectors (log-sum-exp, D): 4 warps x 2 buffers x 2 x 128 floats.
+  static constexpr uint32_t kVecOff = kRingOff + kStages * 2 * kTileBytes;
+  // Fused kernel: dS^T of one 64-query half (128 key rows x 128 B, 128-byte
+  // swizzle), the B operand of dQ^T = K^T dS^T.
+  static constexpr uint32_t kDsOff = kVecOff + 4 * 2 * 2 * kTile * 4;
+  static constexpr uint32_t kDsBytes = kTile * kHalf * 2;
+  static constexpr uint32_t kBarOff = kDsOff + kDsBytes;
   static constexpr int kFixFull = 0;
   static constexpr int kFixEmpty = 1;
   static constexpr int kRingFull = 2;
@@ -219,12 +243,19 @@ struct BwdSmem {
   static constexpr int kAccDone = kPFull + 2;
   static constexpr int kAccFree = kAccDone + 1;
   static constexpr int kFin = kAccFree + 1;
-  static constexpr int kNumBars = kFin + 1;
+  static constexpr int kDqFull = kFin + 1;    // two: dQ^T of a half is in TMEM
+  static constexpr int kDqFree = kDqFull + 2; // two: the dQ warps have read it
+  static constexpr int kDsFree = kDqFree + 2; // the dQ^T product has read the staged dS^T
+  static constexpr int kNumBars = kDsFree + 1;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
+  static_assert(kDsOff % 1024 == 0, "swizzled dS^T tile alignment");
+  static_assert(kAlloc <= 232448, "shared memory per CTA");
   // TMEM columns: two buffers of 64-wide score halves, each S (or S^T) then
-  // dP (or dP^T), then the accumulators.
+  // dP (or dP^T), then the accumulators.  The key-tile kernel writes P^T and
+  // dS^T (bf16, 32 columns each) over the S^T half, which leaves the dP^T half
+  // free for the fused kernel's dQ^T of that half (64 fp32 columns).
   static constexpr uint32_t kColAcc0 = 256, kColAcc1 = 256 + D;
   static __device__ __forceinline__ uint32_t col_s(int h) { return h * 128; }
   static __device__ __forceinline__ uint32_t col_p(int h) { return h * 128 + 64; }
@@ -567,12 +598,19 @@ __device__ __forceinline__ void dkv_loader(const BwdParams& p, uint32_t sbase, c
   if (fix_issued > 0) w.drain(bar(L::kFixFull), (fix_issued - 1) & 1, code | L::kFixFull);
 }
 
-template <int D>
+template <int D, bool kFused>
 __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w) {
   using L = BwdSmem<D>;
+  static_assert(!kFused || D == 128, "the fused dQ^T product has M = d = 128");
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
   constexpr uint32_t idesc_ss = idesc_bf16_f32(kTile, kHalf, false);  // 128 keys x 64 queries
   constexpr uint32_t idesc_ts = idesc_bf16_f32(kTile, D, true);
+  // dQ^T (d x 64 queries) = K^T dS^T: A = the K tile read MN-major (d is its
+  // contiguous axis), B = the staged dS^T, MN-major (queries contiguous).
+  constexpr uint32_t idesc_dq = idesc_bf16_f32(D, kHalf, true) | (1u << 15);
+  const uint64_t kt_desc = mnmajor_desc<D>(sbase + L::kFixOff);
+  const uint64_t ds_desc = smem_desc_sw128(sbase + L::kDsOff, L::kChunkBytes, 1024);
+  uint32_t dq_cnt[2] = {0, 0};  // dQ^T products issued, per half
   const uint32_t t_dv = tmem + L::kColAcc0, t_dk = tmem + L::kColAcc1;
   const uint64_t k_desc = kmajor_desc<D>(sbase + L::kFixOff);
   const uint64_t v_desc = kmajor_desc<D>(sbase + L::kFixOff + L::kTileBytes);
@@ -587,13 +625,25 @@ __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint
     if (h) ++p_cnt1; else ++p_cnt0;
     if (first && items > 0 && !w.wait_warp(bar(L::kAccFree), (items - 1) & 1, code | L::kAccFree)) return false;
     tc_fence_after_sync();
+    if constexpr (kFused) {
+      // dQ^T_h over this tile's 128 keys, into the dP^T columns of half h.  It goes
+      // ahead of dV and dK so that the dQ warps read it out while those execute:
+      // the next S^T into these columns waits for that read.
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_bf16_ss_elect(tmem + L::col_p(h), kt_desc + ((kk * 2048) >> 4), ds_desc + ((kk * 2048) >> 4), idesc_dq,
+                          kk > 0 ? 1u : 0u);
+      tc_commit_elect(bar(L::kDqFull + h));
+      tc_commit_elect(bar(L::kDsFree));
+      ++dq_cnt[h];
+    }
     const uint32_t qaddr = sbase + L::kRingOff + slot * 2 * L::kTileBytes + h * kHalf * 128;
     const uint64_t qb = mnmajor_desc<D>(qaddr), dob = mnmajor_desc<D>(qaddr + L::kTileBytes);
 #pragma unroll
     for (int kk = 0; kk < kHalf / 16; ++kk) {
       const uint32_t acc = (kk > 0 || !first) ? 1u : 0u;
       mma_bf16_ts_elect(t_dv, tmem + L::col_s(h) + kk * 8, dob + ((kk * 2048) >> 4), idesc_ts, acc);
-      mma_bf16_ts_elect(t_dk, tmem + L::col_p(h) + kk * 8, qb + ((kk * 2048) >> 4), idesc_ts, acc);
+      mma_bf16_ts_elect(t_dk, tmem + L::col_s(h) + 32 + kk * 8, qb + ((kk * 2048) >> 4), idesc_ts, acc);
     }
     return true;
   };
@@ -613,6 +663,15 @@ __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint
       tc_fence_after_sync();
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
+        if constexpr (kFused) {
+          // The dQ warps have read the previous dQ^T_h out of these columns.
+          if (dq_cnt[h] > 0 &&
+              !w.wait_warp(bar(L::kDqFree + h), (dq_cnt[h] - 1) & 1, code | (L::kDqFree + h))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+        }
         // S^T_h = K Q_h^T and dP^T_h = V dO_h^T (queries 64h .. 64h+63 of the tile).
         const uint64_t q_desc = kmajor_desc<D>(qaddr + h * kHalf * 128);
         const uint64_t do_desc = kmajor_desc<D>(qaddr + L::kTileBytes + h * kHalf * 128);
@@ -623,7 +682,7 @@ __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint
           mma_bf16_ss_elect(tmem + L::col_p(h), v_desc + off, do_desc + off, idesc_ss, kk > 0 ? 1u : 0u);
         }
         tc_commit_elect(bar(L::kSFull + h));
-        if (s == it.steps - 1 && h == 1) tc_commit_elect(bar(L::kFixEmpty));  // K, V read
+        if (!kFused && s == it.steps - 1 && h == 1) tc_commit_elect(bar(L::kFixEmpty));  // K, V read
         if (h == 1 || s > 0) {
           if (!issue_dkv(1 - h, h == 1 ? slot : prev_slot, first)) {
             ok = false;
@@ -637,12 +696,13 @@ __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint
     }
     if (!ok) break;
     if (!issue_dkv(1, prev_slot, first)) break;  // the item's last half
+    if (kFused) tc_commit_elect(bar(L::kFixEmpty));  // K (read by the dQ^T products too), V
     tc_commit_elect(bar(L::kRingEmpty + prev_slot));
     tc_commit_elect(bar(L::kAccDone));
   }
 }
 
-template <int D>
+template <int D, bool kFused>
 __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w,
                                          int warp, int lane) {
   using L = BwdSmem<D>;
@@ -650,14 +710,30 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
   const int r = warp * 32 + lane;  // key row of the tile = TMEM lane
   const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t t_dv = tmem + lane_bits + L::kColAcc0, t_dk = tmem + lane_bits + L::kColAcc1;
-  // This warp's copy of the step's log2-scaled LSE and D of the 128 query
-  // rows, both negated (they are subtracted).
-  float* s_lse = reinterpret_cast<float*>(__cvta_shared_to_generic(sbase + L::kVecOff)) + warp * 2 * kTile;
-  float* s_dlt = s_lse + kTile;
+  // This warp's two buffers of a step's per-query vectors: the log-sum-exp and D
+  // of the 128 query rows, copied in (zero past the sequence) while the step
+  // before is computed, then negated in place (the LSE also scaled by log2 e).
+  const uint32_t vec_saddr = sbase + L::kVecOff + warp * 4 * kTile * 4;
+  float* const vec_base = reinterpret_cast<float*>(__cvta_shared_to_generic(vec_saddr));
+  auto fetch_vectors = [&](int b, int hq, int m, uint32_t buf) {
+    const size_t bhq = (static_cast<size_t>(b) * p.Hq + hq) * p.N;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int c = lane + 32 * t, q = m * kTile + c;
+      const bool in = q < p.N;
+      const size_t idx = bhq + (in ? q : 0);
+      const uint32_t dst = vec_saddr + (buf * 2 * kTile + c) * 4;
+      cp_async_4(dst, p.lse + idx, in ? 4u : 0u);
+      cp_async_4(dst + kTile * 4, p.delta + idx, in ? 4u : 0u);
+    }
+    cp_async_commit();
+  };
   const float c2 = p.scale_log2;
   const uint64_t c2x2 = f32x2_pack(c2, c2);
   const int code = (kBKernelDkdv << 12) | (kBRoleElem << 8);
   uint32_t s_cnt = 0;
+  uint32_t ds_cnt = 0;  // fused kernel: dS^T halves staged in shared memory
+  bool fetched = false;  // the next step's vectors are already on their way
   int items = 0;
   for (int i = blockIdx.x; i < p.num_items; i += gridDim.x, ++items) {
     const DkvItem it = dkv_item(p, i);
@@ -666,16 +742,33 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
     for (int s = 0; s < it.steps && ok; ++s, ++s_cnt) {
       int hq, m;
       dkv_step(p, it, s, hq, m);
+      const uint32_t buf = s_cnt & 1;
+      float* const s_lse = vec_base + buf * 2 * kTile;
+      float* const s_dlt = s_lse + kTile;
       {
-        const size_t bhq = (static_cast<size_t>(it.b) * p.Hq + hq) * p.N;
-        __syncwarp();  // the previous step's reads of this warp's copy are done
+        if (!fetched) fetch_vectors(it.b, hq, m, buf);
+        cp_async_wait_all();
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          const int c = lane + 32 * t, q = m * kTile + c;
-          s_lse[c] = (q < p.N) ? -p.lse[bhq + q] * kLog2e : 0.f;
-          s_dlt[c] = (q < p.N) ? -p.delta[bhq + q] : 0.f;
+          const int c = lane + 32 * t;
+          s_lse[c] = -s_lse[c] * kLog2e;
+          s_dlt[c] = -s_dlt[c];
         }
-        __syncwarp();
+        __syncwarp();  // every lane's entries are in place; the other buffer's last reads are done
+        // Start the next step's copies (the next item's first step after the last one).
+        fetched = false;
+        if (s + 1 < it.steps) {
+          int hq2, m2;
+          dkv_step(p, it, s + 1, hq2, m2);
+          fetch_vectors(it.b, hq2, m2, buf ^ 1);
+          fetched = true;
+        } else if (i + static_cast<int>(gridDim.x) < p.num_items) {
+          const DkvItem nx = dkv_item(p, i + gridDim.x);
+          int hq2, m2;
+          dkv_step(p, nx, 0, hq2, m2);
+          fetch_vectors(nx.b, hq2, m2, buf ^ 1);
+          fetched = true;
+        }
       }
       const bool partial = block_is_partial(p, m, it.n);
 #pragma unroll 1
@@ -683,6 +776,14 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
         if (!w.wait_warp(bar(L::kSFull + h), s_cnt & 1, code | (L::kSFull + h))) {
           ok = false;
           break;
+        }
+        if constexpr (kFused) {
+          // The staged dS^T is rewritten below: the previous dQ^T product must have read it.
+          if (ds_cnt > 0 && !w.wait_warp(bar(L::kDsFree), (ds_cnt - 1) & 1, code | L::kDsFree)) {
+            ok = false;
+            break;
+          }
+          ++ds_cnt;
         }
         tc_fence_after_sync();
         // Query columns of this half that see the key: lo_c <= c <= hi_c
@@ -725,12 +826,22 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
             dk[chunk][e >> 1] = bf16x2_rn(d0, d1);
           }
         }
-        // P^T and dS^T (bf16, 32 columns each) over the first halves of this
-        // half's S^T and dP^T columns.
+        if constexpr (kFused) {
+          // Stage dS^T for dQ^T = K^T dS^T: this key's row of 64 queries is 128 B
+          // (eight 16-byte chunks, chunk c stored at c ^ (row & 7): the 128-byte
+          // swizzle of an MN-major operand).
+          const uint32_t row_addr = sbase + L::kDsOff + r * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_shared_v4(row_addr + ((c ^ (r & 7)) << 4), dk[c >> 2][(c & 3) * 4], dk[c >> 2][(c & 3) * 4 + 1],
+                         dk[c >> 2][(c & 3) * 4 + 2], dk[c >> 2][(c & 3) * 4 + 3]);
+          fence_proxy_async_smem();
+        }
+        // P^T and dS^T (bf16, 32 columns each) over this half's S^T columns.
         tmem_store_16cols(t_s, pk[0]);
         tmem_store_16cols(t_s + 16, pk[1]);
-        tmem_store_16cols(t_p, dk[0]);
-        tmem_store_16cols(t_p + 16, dk[1]);
+        tmem_store_16cols(t_s + 32, dk[0]);
+        tmem_store_16cols(t_s + 48, dk[1]);
         tmem_store_wait();
         tc_fence_before_sync();
         __syncwarp();
@@ -748,12 +859,80 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
     __syncwarp();
     if (lane == 0) mbar_arrive(bar(L::kAccFree));
   }
+  cp_async_wait_all();  // no copy into shared memory outlives the CTA (a run that stopped early)
   tmem_store_wait();
 }
 
+// Fused kernel, warps 6-9: after each dQ^T_h product, read it out of TMEM
+// (thread = TMEM lane = column c of dQ, 64 query values) and add it into the
+// fp32 accumulator: for each query, the warp's 32 lanes add 32 consecutive
+// floats (one 128-byte reduction).
+template <int D>
+__device__ __forceinline__ void dkv_dq(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w,
+                                       int warp, int lane) {
+  using L = BwdSmem<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  const int quarter = warp & 3;  // TMEM lanes this warp may read
+  const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
+  const int col = quarter * 32 + lane;
+  const int code = (kBKernelFused << 12) | (kBRoleDq << 8);
+  uint32_t cnt[2] = {0, 0};
+  bool ok = true;
+  for (int i = blockIdx.x; ok && i < p.num_items; i += gridDim.x) {
+    const DkvItem it = dkv_item(p, i);
+    for (int s = 0; s < it.steps && ok; ++s) {
+      int hq, m;
+      dkv_step(p, it, s, hq, m);
+      float* head_base = p.dq_acc + (static_cast<size_t>(it.b) * p.Hq + hq) * p.N * D + col;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        if (!w.wait_warp(bar(L::kDqFull + h), cnt[h] & 1, code | (L::kDqFull + h))) {
+          ok = false;
+          break;
+        }
+        ++cnt[h];
+        tc_fence_after_sync();
+        uint32_t a[32], b[32];
+        tmem_load_2x32cols(tmem + lane_bits + L::col_p(h), tmem + lane_bits + L::col_p(h) + 32, a, b);
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::kDqFree + h));
+        const int q0 = m * kTile + h * kHalf;
+        const int nq = min(kHalf, p.N - q0);  // queries of this half inside the sequence
+        float* dst = head_base + static_cast<size_t>(q0) * D;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nq) atomicAdd(dst + static_cast<size_t>(j) * D, __uint_as_float(a[j]));
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (32 + j < nq) atomicAdd(dst + static_cast<size_t>(32 + j) * D, __uint_as_float(b[j]));
+      }
+    }
+  }
+}
+
+// dq = bf16(scale * the fp32 accumulator), eight elements per thread per
+// iteration (two 16-byte loads, one 16-byte store), grid-stride.
+__global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* __restrict__ acc,
+                                                                 __nv_bfloat16* __restrict__ dq, float scale,
+                                                                 int64_t groups8) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < groups8; g += stride) {
+    const float4 x = reinterpret_cast<const float4*>(acc)[2 * g];
+    const float4 y = reinterpret_cast<const float4*>(acc)[2 * g + 1];
+    reinterpret_cast<uint4*>(dq)[g] = make_uint4(bf16x2_rn(x.x * scale, x.y * scale), bf16x2_rn(x.z * scale, x.w * scale),
+                                                 bf16x2_rn(y.x * scale, y.y * scale), bf16x2_rn(y.z * scale, y.w * scale));
+  }
+}
+
 // ------------------------------------------------------------------ entry
+template <int KIND>
+constexpr int bwd_threads() {
+  return KIND == kBKernelFused ? kBwdThreadsFused : kBwdThreads;
+}
+
 template <int D, int KIND>
-__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(bwd_threads<KIND>(), 1) __maxnreg__(KIND == kBKernelFused ? 200 : 255) attn_bwd_kernel(const __grid_constant__ BwdParams p) {
   using L = BwdSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -777,6 +956,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
     mbar_init(bar(L::kAccDone), 1);
     mbar_init(bar(L::kAccFree), 4);  // one arrival per elementwise warp
     mbar_init(bar(L::kFin), 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(bar(L::kDqFull + h), 1);
+      mbar_init(bar(L::kDqFree + h), 4);  // one arrival per dQ warp
+    }
+    mbar_init(bar(L::kDsFree), 1);
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -791,8 +975,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
   const uint32_t tmem = *tmem_slot;
   const BwdWaiter w{p.timeout_ns, abort_flag, p.err};
   if (warp < 4) {
-    if (KIND == kBKernelDq) dq_elem<D>(p, sbase, tmem, w, warp, lane);
-    else dkv_elem<D>(p, sbase, tmem, w, warp, lane);
+    if constexpr (KIND == kBKernelDq) dq_elem<D>(p, sbase, tmem, w, warp, lane);
+    else dkv_elem<D, KIND == kBKernelFused>(p, sbase, tmem, w, warp, lane);
+  } else if (warp >= kBwdDqWarp0) {
+    if constexpr (KIND == kBKernelFused) dkv_dq<D>(p, sbase, tmem, w, warp, lane);
   } else if (warp == kBwdLoaderWarp) {
     if (lane == 0) {
       if (KIND == kBKernelDq) dq_loader<D>(p, sbase, w);
@@ -800,8 +986,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
     }
     __syncwarp();
   } else if (warp == kBwdMmaWarp) {
-    if (KIND == kBKernelDq) dq_mma<D>(p, sbase, tmem, w);
-    else dkv_mma<D>(p, sbase, tmem, w);
+    if constexpr (KIND == kBKernelDq) dq_mma<D>(p, sbase, tmem, w);
+    else dkv_mma<D, KIND == kBKernelFused>(p, sbase, tmem, w);
     // Every MMA this warp issued must complete before TMEM is freed.
     tc_commit_elect(sbase + L::kBarOff + 8u * L::kFin);
     w.drain(sbase + L::kBarOff + 8u * L::kFin, 0, (KIND << 12) | (kBRoleMma << 8) | L::kFin);

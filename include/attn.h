@@ -112,6 +112,10 @@ typedef struct {
                                (and, with a window, j > i + key_offset - window), e.g. a query
                                block against an earlier key block in ring attention; rows that
                                see no key end with out 0 and lse -inf. 0 = the square masks */
+  int bwd_deterministic;    /* backward, d = 128: 1 = the two-kernel path (query-tile dQ kernel,
+                               key-tile dK/dV kernel; seven matmuls per pair, dq bitwise
+                               reproducible, workspace 4 B Hq N bytes, 4-byte aligned);
+                               0 = the fused key-tile kernel (default) */
 } attn_fwd_options;
 
 /* attn_fwd with options (same arguments, same checks); opts may be NULL. */
@@ -247,10 +251,21 @@ int64_t attn_fwd_num_work_items(int64_t B, int64_t Hq, int64_t Hkv, int64_t N, i
  *   dout       device pointer, bf16, [B, Hq, N, d], contiguous, 16-byte aligned
  *   dq         device pointer, bf16, [B, Hq,  N, d], 16-byte aligned; fully overwritten
  *   dk, dv     device pointers, bf16, [B, Hkv, N, d], 16-byte aligned; fully overwritten
- *   workspace  device pointer, 4-byte aligned, at least attn_bwd_workspace_bytes(B, Hq, N)
- *              bytes, owned by the caller; holds D (fp32 [B, Hq, N]) between the kernels
- *              of one call, so it must not be reused until the stream has passed the call
+ *   workspace  device pointer owned by the caller; attn_bwd_workspace_bytes(B, Hq, N) bytes,
+ *              16-byte aligned, always suffice. The minimum: for d = 64 (and d = 128 with
+ *              attn_bwd_ex's bwd_deterministic) 4 B Hq N bytes, 4-byte aligned, holding D
+ *              (fp32 [B, Hq, N]); otherwise the full size, 16-byte aligned: D, then (from
+ *              the next 256-byte boundary) an fp32 [B, Hq, N, 128] dQ accumulator that the
+ *              call zeroes and fills. Not to be reused until the stream has passed the call.
  *   B, Hq, Hkv, N, d, scale, mask_kind, window, stream: as attn_fwd
+ *
+ * Launches: D, then for d = 128 a fused kernel that forms P and dS once per (query, key)
+ * pair (one CTA per 128-key tile: dK, dV in TMEM; dQ's partial sums of each tile added
+ * into the accumulator with fp32 global reductions) and a kernel rounding dQ to bf16; for
+ * d = 64 a query-tile kernel for dQ and a key-tile kernel for dK, dV. With d = 128 the
+ * order of the fp32 additions into dQ varies from run to run, so dq is reproducible only
+ * up to the rounding of those sums (dk and dv are bitwise reproducible); attn_bwd_ex with
+ * bwd_deterministic = 1 runs d = 128 on the two-kernel path instead.
  *
  * The library allocates nothing. Outputs and the workspace must not overlap each other
  * or the inputs (ATTN_ERR_INVALID_ARG). Errors and bounded waits as attn_fwd; a wait
@@ -261,15 +276,16 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* out, const
              int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
              float scale, int mask_kind, int64_t window, cudaStream_t stream);
 
-/* attn_bwd with options (wait bound and CTA count as for attn_fwd_ex; the other fields
-   are ignored); opts may be NULL. */
+/* attn_bwd with options (wait bound and CTA count as for attn_fwd_ex, and
+   bwd_deterministic; the other fields are ignored); opts may be NULL. */
 int attn_bwd_ex(const void* q, const void* k, const void* v, const void* out, const float* lse,
                 const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
                 int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
                 float scale, int mask_kind, int64_t window, cudaStream_t stream,
                 const attn_fwd_options* opts);
 
-/* Workspace bytes attn_bwd needs (4 * B * Hq * N); 0 for invalid sizes. */
+/* Workspace bytes attn_bwd needs for any supported d: 4 B Hq N rounded up to 256, plus
+   4 B Hq N 128 (the d = 128 dQ accumulator); 0 for invalid sizes or a total beyond 2^61. */
 size_t attn_bwd_workspace_bytes(int64_t B, int64_t Hq, int64_t N);
 
 /* attn_debug_error for the backward kernels' error word (same contract). */

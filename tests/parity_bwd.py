@@ -54,18 +54,18 @@ def bounds(q, k, v, do, scale, mask_kind, window):
     return bq, bk, bv
 
 
-def run_cuda_bwd(q, k, v, do, mask, window=None, scale=None):
+def run_cuda_bwd(q, k, v, do, mask, window=None, scale=None, deterministic=False):
     from exact_io_aware_72_b200 import bwd, fwd
     out, lse = fwd(q, k, v, scale=scale, mask=mask, window=window)
-    dq, dk, dv = bwd(q, k, v, out, lse, do, scale=scale, mask=mask, window=window)
+    dq, dk, dv = bwd(q, k, v, out, lse, do, scale=scale, mask=mask, window=window, deterministic=deterministic)
     torch.cuda.synchronize()
     return dq, dk, dv
 
 
-def check_bwd_case(B, Hq, Hkv, N, d, mask, window=None, seed=0, scale=None, sharp=False):
+def check_bwd_case(B, Hq, Hkv, N, d, mask, window=None, seed=0, scale=None, sharp=False, deterministic=False):
     q, k, v = make_qkv(B, Hq, Hkv, N, d, seed, device="cpu", sharp=sharp)
     do = make_dout(B, Hq, N, d, seed)
-    got = run_cuda_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), mask, window, scale)
+    got = run_cuda_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), mask, window, scale, deterministic)
     qn, kn, vn, don = to_np(q), to_np(k), to_np(v), to_np(do)
     s = (1.0 / np.sqrt(d)) if scale is None else scale
     kind = MASK_NAMES[mask]

@@ -113,7 +113,9 @@ def call_bwd(lib, q=Q, k=K, v=V, o=O, l=L, do=DO, dq=DQ, dk=DK, dv=DV, ws=WS, ws
 
 
 def test_backward_workspace_bytes(lib):
-    assert lib.attn_bwd_workspace_bytes(2, 32, 8192) == 4 * 2 * 32 * 8192
+    rows = 2 * 32 * 8192
+    assert lib.attn_bwd_workspace_bytes(2, 32, 8192) == 4 * rows + 4 * rows * 128   # D, then the dQ sums
+    assert lib.attn_bwd_workspace_bytes(1, 1, 3) == 256 + 4 * 3 * 128                # the sums start 256-aligned
     assert lib.attn_bwd_workspace_bytes(0, 1, 1) == 0 and lib.attn_bwd_workspace_bytes(1, 1, -1) == 0
     assert lib.attn_bwd_workspace_bytes(1 << 30, 1 << 30, 1 << 30) == 0   # beyond 63 bits
 
@@ -138,7 +140,29 @@ def test_backward_valid_arguments_reach_the_device_check(lib):
     if torch.cuda.is_available():
         pytest.skip("GPU present")
     assert call_bwd(lib) == 4
-    assert call_bwd(lib, d=128, mask=2, window=10 ** 9) == 4
+    ws = lib.attn_bwd_workspace_bytes(1, 2, 256)
+    assert call_bwd(lib, d=128, mask=2, window=10 ** 9, ws_bytes=ws) == 4
+    # d = 128 needs the dQ accumulator and a 16-byte aligned workspace
+    assert call_bwd(lib, d=128, ws_bytes=ws - 4) == 1
+    assert call_bwd(lib, d=128, ws_bytes=ws, ws=WS + 4) == 3
+
+
+def test_backward_deterministic_option_needs_only_the_row_terms(lib):
+    """attn_bwd_ex with bwd_deterministic takes d = 128 down the two-kernel path, whose
+    workspace is D alone (4 B Hq N bytes, 4-byte aligned)."""
+    import ctypes
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    opts = A.FwdOptions(0, 0, 0)
+    opts.bwd_deterministic = 1
+
+    def call(ws, ws_bytes, o):
+        return lib.attn_bwd_ex(Q, K, V, O, L, DO, DQ, DK, DV, ws, ws_bytes, 1, 2, 2, 256, 128, 0.125, 1, 0, None,
+                               ctypes.byref(o) if o is not None else None)
+    assert call(WS + 4, 4 * 2 * 256, opts) == 4          # valid: reaches the device check
+    assert call(WS + 4, 4 * 2 * 256, None) in (1, 3)     # the fused default needs more, aligned
+    assert call(WS, 4 * 2 * 256 - 4, opts) == 1
 
 
 # ------------------------------------------------------------------ decoding
