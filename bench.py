@@ -60,8 +60,8 @@ KERNEL_SOURCES = ["exact_io_aware_72_b200/csrc/attn_fwd.cu", "exact_io_aware_72_
 # long workload's figure is the capture of the same kernel on a causal
 # N = 32768 case (1, 32, 32, 32768, 128) times 4: DRAM bytes grow linearly in N.
 NCU_TRAFFIC = {
-    ("dense", "59529aafc8fdc7bc"): 408637696 + 110999296,
-    ("long", "59529aafc8fdc7bc"): 4 * (904199936 + 251104512),
+    ("dense", "e2664b285cb35e2b"): 410178304 + 111494656,
+    ("long", "e2664b285cb35e2b"): 4 * (937351680 + 253613312),
 }
 
 
@@ -492,7 +492,7 @@ def run_backward(args, w):
     out, lse = fwd(q, k, v, scale=w.scale, mask=w.mask, window=w.window)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     det = bool(args.bwd_deterministic)
-    fused = w.d == 128 and not det
+    fused = w.d == 128 and w.Hq == w.Hkv and not det
     ws_bytes = int(load_library().attn_bwd_workspace_bytes(w.B, w.Hq, w.N)) if fused else 4 * w.B * w.Hq * w.N
     ws = torch.empty(ws_bytes // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)

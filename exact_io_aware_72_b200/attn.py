@@ -222,9 +222,9 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, ls
 
     ``out`` and ``lse`` are the forward's outputs for these inputs. The fp32
     workspace (allocated here when not given) holds the row terms
-    D = rowsum(dout * out) and, for d = 128, the fp32 sums of dq: B*Hq*N floats
-    for d = 64 or ``deterministic``, ``attn_bwd_workspace_bytes(B, Hq, N)`` bytes
-    for d = 128.  ``deterministic`` runs d = 128 on the two-kernel path (dq bitwise
+    D = rowsum(dout * out) and, on the fused path (d = 128, Hq == Hkv), the fp32
+    sums of dq: ``attn_bwd_workspace_bytes(B, Hq, N)`` bytes there, B*Hq*N floats
+    otherwise.  ``deterministic`` takes the two-kernel path there too (dq bitwise
     reproducible; seven matmuls per pair instead of five).
     """
     lib = load_library()
@@ -247,7 +247,7 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, ls
         _check(t, name, torch.bfloat16, 4)
         if t.shape != ref.shape:
             raise ValueError(f"{name} has the wrong shape")
-    fused = d == 128 and not deterministic
+    fused = d == 128 and Hq == Hkv and not deterministic  # the library's choice of path
     ws_bytes = int(lib.attn_bwd_workspace_bytes(B, Hq, N)) if fused else 4 * B * Hq * N
     if workspace is None:
         workspace = torch.empty(ws_bytes // 4, dtype=torch.float32, device=q.device)

@@ -156,7 +156,10 @@ int attn_bwd_ex(const void* q, const void* k, const void* v, const void* out, co
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   // Byte counts must fit in 63 bits (B * Hq * N <= 2^60 after sizes_ok).
   if (B * Hq * N > (int64_t(1) << 61) / (d * 4)) return ATTN_ERR_INVALID_ARG;
-  const bool fused = (d == 128) && !(opts && opts->bwd_deterministic);
+  // The fused kernel where each KV head serves one query head. With grouped heads a key
+  // tile's dQ partial sums go to every query head of its group, whose fp32 accumulators
+  // (and Q, dO) then outgrow L2; there the two-kernel path measured faster.
+  const bool fused = (d == 128) && Hq == Hkv && !(opts && opts->bwd_deterministic);
   const size_t ws = bwd_workspace_bytes(B, Hq, N, fused ? 128 : 0);
   if (ws == 0 || workspace_bytes < ws) return ATTN_ERR_INVALID_ARG;
   const size_t q_bytes = static_cast<size_t>(B * Hq * N * d) * 2;

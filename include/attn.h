@@ -115,7 +115,7 @@ typedef struct {
   int bwd_deterministic;    /* backward, d = 128: 1 = the two-kernel path (query-tile dQ kernel,
                                key-tile dK/dV kernel; seven matmuls per pair, dq bitwise
                                reproducible, workspace 4 B Hq N bytes, 4-byte aligned);
-                               0 = the fused key-tile kernel (default) */
+                               0 = the fused key-tile kernel where Hq == Hkv (default) */
 } attn_fwd_options;
 
 /* attn_fwd with options (same arguments, same checks); opts may be NULL. */
@@ -252,20 +252,21 @@ int64_t attn_fwd_num_work_items(int64_t B, int64_t Hq, int64_t Hkv, int64_t N, i
  *   dq         device pointer, bf16, [B, Hq,  N, d], 16-byte aligned; fully overwritten
  *   dk, dv     device pointers, bf16, [B, Hkv, N, d], 16-byte aligned; fully overwritten
  *   workspace  device pointer owned by the caller; attn_bwd_workspace_bytes(B, Hq, N) bytes,
- *              16-byte aligned, always suffice. The minimum: for d = 64 (and d = 128 with
- *              attn_bwd_ex's bwd_deterministic) 4 B Hq N bytes, 4-byte aligned, holding D
- *              (fp32 [B, Hq, N]); otherwise the full size, 16-byte aligned: D, then (from
+ *              16-byte aligned, always suffice. The minimum: on the two-kernel path (d = 64,
+ *              Hq != Hkv, or bwd_deterministic) 4 B Hq N bytes, 4-byte aligned, holding D
+ *              (fp32 [B, Hq, N]); on the fused path the full size, 16-byte aligned: D, then (from
  *              the next 256-byte boundary) an fp32 [B, Hq, N, 128] dQ accumulator that the
  *              call zeroes and fills. Not to be reused until the stream has passed the call.
  *   B, Hq, Hkv, N, d, scale, mask_kind, window, stream: as attn_fwd
  *
- * Launches: D, then for d = 128 a fused kernel that forms P and dS once per (query, key)
- * pair (one CTA per 128-key tile: dK, dV in TMEM; dQ's partial sums of each tile added
- * into the accumulator with fp32 global reductions) and a kernel rounding dQ to bf16; for
- * d = 64 a query-tile kernel for dQ and a key-tile kernel for dK, dV. With d = 128 the
- * order of the fp32 additions into dQ varies from run to run, so dq is reproducible only
- * up to the rounding of those sums (dk and dv are bitwise reproducible); attn_bwd_ex with
- * bwd_deterministic = 1 runs d = 128 on the two-kernel path instead.
+ * Launches: D, then for d = 128 with Hq == Hkv a fused kernel that forms P and dS once
+ * per (query, key) pair (one CTA per 128-key tile: dK, dV in TMEM; dQ's partial sums of
+ * each tile added into the accumulator with fp32 global reductions) and a kernel rounding
+ * dQ to bf16; otherwise (d = 64, grouped heads) a query-tile kernel for dQ and a key-tile
+ * kernel for dK, dV. On the fused path the order of the fp32 additions into dQ varies
+ * from run to run, so dq is reproducible only up to the rounding of those sums (dk and dv
+ * are bitwise reproducible); attn_bwd_ex with bwd_deterministic = 1 takes the two-kernel
+ * path there too.
  *
  * The library allocates nothing. Outputs and the workspace must not overlap each other
  * or the inputs (ATTN_ERR_INVALID_ARG). Errors and bounded waits as attn_fwd; a wait

@@ -33,6 +33,12 @@ def test_head_sharing(cuda_ok, shape, mask, window):
     check_bwd_case(B, Hq, Hkv, N, 128, mask, window, seed=sum(shape))
 
 
+@pytest.mark.parametrize("w", [1, 127, 129, 300])
+def test_fused_path_windows(cuda_ok, w):
+    """The fused d = 128 path (Hq == Hkv) under sliding windows, ragged N, B > 1."""
+    check_bwd_case(2, 2, 2, 700, 128, "sliding_window", window=w, seed=40 + w)
+
+
 @pytest.mark.parametrize("mask,window", [("causal", None), ("full", None), ("sliding_window", 200)])
 def test_deterministic_path_d128(cuda_ok, mask, window):
     """The two-kernel path that bwd_deterministic selects for d = 128, ragged and multi-tile,
@@ -46,8 +52,8 @@ def test_fused_and_deterministic_agree(cuda_ok):
     forms them), dq close (the two paths form dS from S and from S^T, whose fp32 sums may
     round differently, and add dQ's terms in different orders; each path meets the
     oracle's bound in the tests above)."""
-    q, k, v = (t.cuda() for t in make_qkv(1, 8, 2, 1500, 128, 33))
-    do = make_dout(1, 8, 1500, 128, 33).cuda()
+    q, k, v = (t.cuda() for t in make_qkv(1, 4, 4, 1500, 128, 33))
+    do = make_dout(1, 4, 1500, 128, 33).cuda()
     a = run_cuda_bwd(q, k, v, do, "causal")
     b = run_cuda_bwd(q, k, v, do, "causal", deterministic=True)
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
@@ -69,8 +75,9 @@ def dq_sum_order_tolerance(dq):
                        torch.frexp(dq.float().abs())[1] - 8) + 2.0 ** -16
 
 
-def test_window_ge_N_is_causal_bitwise(cuda_ok):
-    q, k, v = (t.cuda() for t in make_qkv(1, 4, 2, 333, 128, 9))
+@pytest.mark.parametrize("hkv", [2, 4])  # grouped heads: two-kernel path; Hq == Hkv: fused
+def test_window_ge_N_is_causal_bitwise(cuda_ok, hkv):
+    q, k, v = (t.cuda() for t in make_qkv(1, 4, hkv, 333, 128, 9))
     do = make_dout(1, 4, 333, 128, 9).cuda()
     ref = run_cuda_bwd(q, k, v, do, "causal")
     for w in (333, 10 ** 6):
@@ -83,9 +90,10 @@ def test_window_ge_N_is_causal_bitwise(cuda_ok):
 def test_repeated_calls_agree(cuda_ok, d, det):
     """Three calls on the same inputs (several key tiles add into each query tile's dQ):
     dk and dv are identical; dq is identical on the two-kernel path (d = 64, or d = 128
-    with deterministic) and within the rounding of its fp32 sums on the fused one."""
-    q, k, v = (t.cuda() for t in make_qkv(1, 8, 2, 1000, d, 21))
-    do = make_dout(1, 8, 1000, d, 21).cuda()
+    with deterministic) and within the rounding of its fp32 sums on the fused one
+    (d = 128, Hq == Hkv)."""
+    q, k, v = (t.cuda() for t in make_qkv(1, 4, 4, 1000, d, 21))
+    do = make_dout(1, 4, 1000, d, 21).cuda()
     ref = run_cuda_bwd(q, k, v, do, "full", deterministic=det)
     for _ in range(2):
         got = run_cuda_bwd(q, k, v, do, "full", deterministic=det)
