@@ -614,7 +614,7 @@ __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint
   const uint32_t t_dv = tmem + L::kColAcc0, t_dk = tmem + L::kColAcc1;
   const uint64_t k_desc = kmajor_desc<D>(sbase + L::kFixOff);
   const uint64_t v_desc = kmajor_desc<D>(sbase + L::kFixOff + L::kTileBytes);
-  const int code = (kBKernelDkdv << 12) | (kBRoleMma << 8);
+  const int code = ((kFused ? kBKernelFused : kBKernelDkdv) << 12) | (kBRoleMma << 8);
   uint32_t n = 0;
   uint32_t p_cnt0 = 0, p_cnt1 = 0;  // P / dS halves consumed, per half
   int items = 0;
@@ -730,7 +730,7 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
   };
   const float c2 = p.scale_log2;
   const uint64_t c2x2 = f32x2_pack(c2, c2);
-  const int code = (kBKernelDkdv << 12) | (kBRoleElem << 8);
+  const int code = ((kFused ? kBKernelFused : kBKernelDkdv) << 12) | (kBRoleElem << 8);
   uint32_t s_cnt = 0;
   uint32_t ds_cnt = 0;  // fused kernel: dS^T halves staged in shared memory
   bool fetched = false;  // the next step's vectors are already on their way
