@@ -59,9 +59,11 @@ KERNEL_SOURCES = ["exact_io_aware_72_b200/csrc/attn_fwd.cu", "exact_io_aware_72_
 # sources it was taken on; reported only while the sources still match.  The
 # long workload's figure is the capture of the same kernel on a causal
 # N = 32768 case (1, 32, 32, 32768, 128) times 4: DRAM bytes grow linearly in N.
+# The FP8 long figure is a capture of the full launch (E4M3 q, k, v: 1.2 GiB).
 NCU_TRAFFIC = {
     ("dense", "e2664b285cb35e2b"): 410178304 + 111494656,
     ("long", "e2664b285cb35e2b"): 4 * (937351680 + 253613312),
+    ("long_fp8", "e2664b285cb35e2b"): 2079931136 + 1068808704,
 }
 
 
