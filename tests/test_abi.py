@@ -161,7 +161,10 @@ def test_backward_deterministic_option_needs_only_the_row_terms(lib):
         return lib.attn_bwd_ex(Q, K, V, O, L, DO, DQ, DK, DV, ws, ws_bytes, 1, 2, 2, 256, 128, 0.125, 1, 0, None,
                                ctypes.byref(o) if o is not None else None)
     assert call(WS + 4, 4 * 2 * 256, opts) == 4          # valid: reaches the device check
-    assert call(WS + 4, 4 * 2 * 256, None) in (1, 3)     # the fused default needs more, aligned
+    assert call(WS + 4, 4 * 2 * 256, None) == 1          # the fused default needs the dQ sums too
+    full = lib.attn_bwd_workspace_bytes(1, 2, 256)
+    assert call(WS + 4, full, None) == 3                 # ... in a 16-byte aligned workspace
+    assert call(WS, full, None) == 4
     assert call(WS, 4 * 2 * 256 - 4, opts) == 1
     # grouped heads take the two-kernel path by default: D alone suffices
     assert lib.attn_bwd_ex(Q, K, V, O, L, DO, DQ, DK, DV, WS + 4, 4 * 4 * 256, 1, 4, 2, 256, 128, 0.125, 1, 0, None,
