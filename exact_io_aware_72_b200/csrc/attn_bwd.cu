@@ -81,7 +81,9 @@ int bwd_device_setup(BwdDevice& out) {
       info.err_word = static_cast<int*>(addr);
       if (set_smem<64, kBKernelDq>() != cudaSuccess || set_smem<64, kBKernelDkdv>() != cudaSuccess ||
           set_smem<128, kBKernelDq>() != cudaSuccess || set_smem<128, kBKernelDkdv>() != cudaSuccess ||
-          set_smem<128, kBKernelFused>() != cudaSuccess)
+          set_smem<128, kBKernelFused>() != cudaSuccess || set_smem<64, kBKernelDkdvFull>() != cudaSuccess ||
+          set_smem<128, kBKernelDkdvFull>() != cudaSuccess || set_smem<64, kBKernelDqFull>() != cudaSuccess ||
+          set_smem<128, kBKernelDqFull>() != cudaSuccess)
         return ATTN_ERR_CUDA;
     }
     info.probed = true;
@@ -249,11 +251,12 @@ int attn_bwd_ex(const void* q, const void* k, const void* v, const void* out, co
   }
   p.num_items = static_cast<int>(B * Hq * p.num_blk);  // dQ: one query tile per item
   int grid = static_cast<int>(std::min<int64_t>(sms, p.num_items));
-  e = (d == 128) ? launch_bwd<128, kBKernelDq>(p, grid, stream) : launch_bwd<64, kBKernelDq>(p, grid, stream);
+  e = (d == 128) ? launch_bwd<128, kBKernelDqFull>(p, grid, stream) : launch_bwd<64, kBKernelDqFull>(p, grid, stream);
   if (e != cudaSuccess) return ATTN_ERR_CUDA;
   p.num_items = static_cast<int>(B * Hkv * p.num_blk);  // dK, dV: one key tile per item
   grid = static_cast<int>(std::min<int64_t>(sms, p.num_items));
-  e = (d == 128) ? launch_bwd<128, kBKernelDkdv>(p, grid, stream) : launch_bwd<64, kBKernelDkdv>(p, grid, stream);
+  e = (d == 128) ? launch_bwd<128, kBKernelDkdvFull>(p, grid, stream)
+                 : launch_bwd<64, kBKernelDkdvFull>(p, grid, stream);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -57,7 +57,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int { kBMaskFull = 0, kBMaskCausal = 1, kBMaskWindow = 2 };
 enum : int { kBRoleLoader = 1, kBRoleMma = 2, kBRoleElem = 3, kBRoleDq = 4 };
-enum : int { kBKernelDq = 0, kBKernelDkdv = 1, kBKernelFused = 2 };
+enum : int { kBKernelDq = 0, kBKernelDkdv = 1, kBKernelFused = 2, kBKernelDkdvFull = 3, kBKernelDqFull = 4 };
 
 struct BwdParams {
   CUtensorMap tm_q;   // [B*Hq, N, d] bf16, box 64 x 128, 128-byte swizzle
@@ -246,7 +246,11 @@ struct BwdSmem {
   static constexpr int kDqFull = kFin + 1;    // two: dQ^T of a half is in TMEM
   static constexpr int kDqFree = kDqFull + 2; // two: the dQ warps have read it
   static constexpr int kDsFree = kDqFree + 2; // the dQ^T product has read the staged dS^T
-  static constexpr int kNumBars = kDsFree + 1;
+  // Full-tile key-tile kernel: a slot's Q and dO tiles land and are released
+  // separately (kRingFull / kRingEmpty then cover Q alone).
+  static constexpr int kRing2Full = kDsFree + 1;
+  static constexpr int kRing2Empty = kRing2Full + kStages;
+  static constexpr int kNumBars = kRing2Empty + kStages;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kBytes = kMiscOff + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
@@ -543,7 +547,10 @@ __device__ __forceinline__ void dkv_step(const BwdParams& p, const DkvItem& it, 
   m = it.qlo + (s - h * per_head);
 }
 
-template <int D>
+// kSplit (the full-tile key-tile kernel): a slot's Q and dO tiles land and are
+// released through their own barriers, so Q can be refilled as soon as the
+// products that read it are done.
+template <int D, bool kSplit>
 __device__ __forceinline__ void dkv_loader(const BwdParams& p, uint32_t sbase, const BwdWaiter& w) {
   using L = BwdSmem<D>;
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
@@ -573,26 +580,37 @@ __device__ __forceinline__ void dkv_loader(const BwdParams& p, uint32_t sbase, c
       int hq, m;
       dkv_step(p, it, s, hq, m);
       const uint32_t slot = n % L::kStages;
+      const uint32_t dst = sbase + L::kRingOff + slot * 2 * L::kTileBytes;
+      const int zq = it.b * p.Hq + hq;
+      const int do_full = kSplit ? L::kRing2Full : L::kRingFull;
       if (n >= (uint32_t)L::kStages &&
           !w.wait(bar(L::kRingEmpty + slot), ((n / L::kStages) - 1) & 1, code | (L::kRingEmpty + slot))) {
         ok = false;
         break;
       }
-      const uint32_t dst = sbase + L::kRingOff + slot * 2 * L::kTileBytes;
-      const int zq = it.b * p.Hq + hq;
-      mbar_arrive_expect_tx(bar(L::kRingFull + slot), 2 * L::kTileBytes);
+      mbar_arrive_expect_tx(bar(L::kRingFull + slot), (kSplit ? 1 : 2) * L::kTileBytes);
 #pragma unroll
-      for (int c = 0; c < L::kChunks; ++c) {
+      for (int c = 0; c < L::kChunks; ++c)
         tma_load_3d(dst + c * L::kChunkBytes, &p.tm_q, bar(L::kRingFull + slot), c * 64, m * kTile, zq, pol_q);
-        tma_load_3d(dst + L::kTileBytes + c * L::kChunkBytes, &p.tm_do, bar(L::kRingFull + slot), c * 64, m * kTile, zq,
-                    pol_q);
+      if constexpr (kSplit) {
+        if (n >= (uint32_t)L::kStages &&
+            !w.wait(bar(L::kRing2Empty + slot), ((n / L::kStages) - 1) & 1, code | (L::kRing2Empty + slot))) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(do_full + slot), L::kTileBytes);
       }
+#pragma unroll
+      for (int c = 0; c < L::kChunks; ++c)
+        tma_load_3d(dst + L::kTileBytes + c * L::kChunkBytes, &p.tm_do, bar(do_full + slot), c * 64, m * kTile, zq,
+                    pol_q);
     }
   }
   for (uint32_t s = 0; s < (uint32_t)L::kStages; ++s) {
     if (n > s) {
       const uint32_t last = s + ((n - 1 - s) / L::kStages) * L::kStages;
       w.drain(bar(L::kRingFull + s), (last / L::kStages) & 1, code | (L::kRingFull + s));
+      if constexpr (kSplit) w.drain(bar(L::kRing2Full + s), (last / L::kStages) & 1, code | (L::kRing2Full + s));
     }
   }
   if (fix_issued > 0) w.drain(bar(L::kFixFull), (fix_issued - 1) & 1, code | L::kFixFull);
@@ -863,6 +881,429 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
   tmem_store_wait();
 }
 
+// ------------------------------------------------------------------ dQ kernel, full tiles
+// The query-tile kernel with whole 128-key products, arranged like the full-tile
+// key-tile kernel: X = [0, 128) holds S = Q K^T; Y = [128, 256) holds dP = dO V^T,
+// then dS (bf16, [128, 192)); dQ after them.  Per key tile g the issuer queues
+//   S(g) -> X        once the elementwise warps have loaded S(g-1) out of X,
+//   dQ += dS(g-1) K  once dS(g-1) is in Y,
+//   dP(g) -> Y       behind it,
+// so the exponentials of tile g run while the tensor core does dQ of tile g-1
+// and dP of tile g.  P is kept as bf16 until dP arrives.
+template <int D>
+__device__ __forceinline__ void dqf_mma(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w) {
+  using L = BwdSmem<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  constexpr int kSFull = L::kSFull, kDpFull = L::kSFull + 1;
+  constexpr int kPFull = L::kPFull, kXFree = L::kPFull + 1;
+  constexpr uint32_t idesc_ss = idesc_bf16_f32(kTile, kTile, false);  // 128 queries x 128 keys
+  constexpr uint32_t idesc_ts = idesc_bf16_f32(kTile, D, true);
+  const uint32_t tX = tmem, tY = tmem + 128, t_acc = tmem + L::kColAcc0;
+  const uint64_t q_desc = kmajor_desc<D>(sbase + L::kFixOff);
+  const uint64_t do_desc = kmajor_desc<D>(sbase + L::kFixOff + L::kTileBytes);
+  const int code = (kBKernelDqFull << 12) | (kBRoleMma << 8);
+  uint32_t g = 0, b_cnt = 0;
+  int acc_items = 0, items = 0;
+  bool ok = true;
+  bool pend = false, pend_first = false, pend_last = false;
+  uint32_t pend_slot = 0;
+  auto issue_b = [&]() -> bool {
+    if (!w.wait_warp(bar(kPFull), b_cnt & 1, code | kPFull)) return false;
+    if (pend_first && acc_items > 0 && !w.wait_warp(bar(L::kAccFree), (acc_items - 1) & 1, code | L::kAccFree))
+      return false;
+    tc_fence_after_sync();
+    const uint64_t kb = mnmajor_desc<D>(sbase + L::kRingOff + pend_slot * 2 * L::kTileBytes);
+#pragma unroll
+    for (int kk = 0; kk < kTile / 16; ++kk)
+      mma_bf16_ts_elect(t_acc, tY + kk * 8, kb + ((kk * 2048) >> 4), idesc_ts, (kk > 0 || !pend_first) ? 1u : 0u);
+    tc_commit_elect(bar(L::kRingEmpty + pend_slot));  // that tile's K (and V, read by its dP) are done
+    if (pend_last) {
+      tc_commit_elect(bar(L::kAccDone));
+      ++acc_items;
+    }
+    ++b_cnt;
+    pend = false;
+    return true;
+  };
+  for (int i = blockIdx.x; ok && i < p.num_items; i += gridDim.x, ++items) {
+    const DqItem it = dq_item(p, i);
+    if (!w.wait_warp(bar(L::kFixFull), items & 1, code | L::kFixFull)) break;
+    tc_fence_after_sync();
+    for (int j = it.lo; j <= it.hi; ++j, ++g) {
+      const uint32_t slot = g % L::kStages;
+      if (!w.wait_warp(bar(L::kRingFull + slot), (g / L::kStages) & 1, code | (L::kRingFull + slot)) ||
+          (g > 0 && !w.wait_warp(bar(kXFree), (g - 1) & 1, code | kXFree))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t kaddr = sbase + L::kRingOff + slot * 2 * L::kTileBytes;
+      const uint64_t k_desc = kmajor_desc<D>(kaddr), v_desc = kmajor_desc<D>(kaddr + L::kTileBytes);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = kmajor_off<D>(kk);
+        mma_bf16_ss_elect(tX, q_desc + off, k_desc + off, idesc_ss, kk > 0 ? 1u : 0u);
+      }
+      tc_commit_elect(bar(kSFull));
+      if (pend && !issue_b()) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = kmajor_off<D>(kk);
+        mma_bf16_ss_elect(tY, do_desc + off, v_desc + off, idesc_ss, kk > 0 ? 1u : 0u);
+      }
+      tc_commit_elect(bar(kDpFull));
+      if (j == it.hi) tc_commit_elect(bar(L::kFixEmpty));  // Q and dO read by the item's last products
+      pend = true;
+      pend_slot = slot;
+      pend_first = (j == it.lo);
+      pend_last = (j == it.hi);
+    }
+  }
+  if (ok && pend) issue_b();
+}
+
+template <int D>
+__device__ __forceinline__ void dqf_elem(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w,
+                                         int warp, int lane) {
+  using L = BwdSmem<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  constexpr int kSFull = L::kSFull, kDpFull = L::kSFull + 1;
+  constexpr int kPFull = L::kPFull, kXFree = L::kPFull + 1;
+  const int r = warp * 32 + lane;  // row of the query tile = TMEM lane
+  const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t tX = tmem + lane_bits, tY = tmem + lane_bits + 128, t_acc = tmem + lane_bits + L::kColAcc0;
+  const float c2 = p.scale_log2;
+  const int code = (kBKernelDqFull << 12) | (kBRoleElem << 8);
+  uint32_t g = 0;
+  int items = 0;
+  for (int i = blockIdx.x; i < p.num_items; i += gridDim.x, ++items) {
+    const DqItem it = dq_item(p, i);
+    const int row = it.m * kTile + r;
+    const bool row_ok = row < p.N;
+    const size_t bhrow = (static_cast<size_t>(it.b) * p.Hq + it.hq) * p.N + (row_ok ? row : 0);
+    const float lse2 = row_ok ? p.lse[bhrow] * kLog2e : 0.f;
+    const float dlt = row_ok ? p.delta[bhrow] : 0.f;
+    const uint64_t c2x2 = f32x2_pack(c2, c2), nlse2x2 = f32x2_pack(-lse2, -lse2), ndlt2 = f32x2_pack(-dlt, -dlt);
+    bool ok = true;
+    for (int j = it.lo; j <= it.hi && ok; ++j, ++g) {
+      if (!w.wait_warp(bar(kSFull), g & 1, code | kSFull)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      uint32_t sv[128];
+      tmem_load_128cols(tX, sv);
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kXFree));
+      if (block_is_partial(p, it.m, j)) {
+        // Visible key columns of this row: lo_c <= c <= hi_c.
+        const int j0 = j * kTile;
+        const int hi_c = row_ok ? min(p.N - 1, p.mask_kind == kBMaskFull ? p.N - 1 : row) - j0 : -1;
+        const int lo_c = (p.mask_kind == kBMaskWindow) ? row - p.window + 1 - j0 : 0;
+#pragma unroll
+        for (int c = 0; c < kTile; ++c)
+          if (c > hi_c || c < lo_c) sv[c] = 0xff800000u;  // -inf
+      }
+      uint32_t pk[kTile / 2];  // P, bf16 pairs of keys
+#pragma unroll
+      for (int c = 0; c < kTile; c += 2) {
+        float x0, x1;
+        f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), c2x2, nlse2x2), x0,
+                     x1);
+        pk[c >> 1] = bf16x2_rn(bexp2(x0), bexp2(x1));
+      }
+      if (!w.wait_warp(bar(kDpFull), g & 1, code | kDpFull)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      uint32_t ds[kTile / 2];
+#pragma unroll
+      for (int chunk = 0; chunk < 4; ++chunk) {
+        uint32_t pv[32];
+        tmem_load_32cols(tY + chunk * 32, pv);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const uint32_t pw = pk[(chunk * 32 + e) >> 1];
+          float d0, d1;
+          f32x2_unpack(f32x2_mul(f32x2_pack(__uint_as_float(pw << 16), __uint_as_float(pw & 0xffff0000u)),
+                                 f32x2_add(f32x2_pack(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1])), ndlt2)),
+                       d0, d1);
+          ds[(chunk * 32 + e) >> 1] = bf16x2_rn(d0, d1);
+        }
+      }
+      // dS over Y's first 64 columns (all of dP has been read).
+      tmem_store_32cols(tY, *reinterpret_cast<const uint32_t(*)[32]>(&ds[0]));
+      tmem_store_32cols(tY + 32, *reinterpret_cast<const uint32_t(*)[32]>(&ds[32]));
+      tmem_store_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kPFull));
+    }
+    if (!ok) break;
+    if (!w.wait_warp(bar(L::kAccDone), items & 1, code | L::kAccDone)) break;
+    tc_fence_after_sync();
+    store_acc_row<D>(t_acc, p.scale, p.dq + bhrow * D, row_ok);
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(L::kAccFree));
+  }
+  tmem_store_wait();
+}
+
+// ------------------------------------------------------------------ dK/dV kernel, full tiles
+// The key-tile kernel with whole 128-query products: S^T and dP^T of a step are
+// single M = 128, N = 128 products (narrower products keep the tensor pipe far
+// from busy), and the elementwise warps still overlap the tensor core.  TMEM:
+// X = [0, 128) holds S^T; Y = [128, 256) holds dP^T, then P^T (bf16, [128, 192))
+// and dS^T ([192, 256)); dV and dK after them.  Per step g the issuer queues
+//   S^T(g) -> X      once the elementwise warps have loaded S^T(g-1) out of X,
+//   dV, dK (g-1)     once P^T(g-1) and dS^T(g-1) are in Y,
+//   dP^T(g) -> Y     behind them (in issue order, so after they read Y),
+// so the exponentials of step g run while the tensor core does dV, dK of step g-1
+// and dP^T of step g.  P is kept as bf16 until dP arrives; dS = P (dP - D) is
+// formed from that bf16 P.
+template <int D>
+__device__ __forceinline__ void dkvf_mma(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w) {
+  using L = BwdSmem<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  constexpr int kSFull = L::kSFull, kDpFull = L::kSFull + 1;  // barrier indices of this kernel
+  constexpr int kPFull = L::kPFull, kXFree = L::kPFull + 1;
+  constexpr uint32_t idesc_ss = idesc_bf16_f32(kTile, kTile, false);  // 128 keys x 128 queries
+  constexpr uint32_t idesc_ts = idesc_bf16_f32(kTile, D, true);
+  const uint32_t tX = tmem, tY = tmem + 128, t_dv = tmem + L::kColAcc0, t_dk = tmem + L::kColAcc1;
+  const uint64_t k_desc = kmajor_desc<D>(sbase + L::kFixOff);
+  const uint64_t v_desc = kmajor_desc<D>(sbase + L::kFixOff + L::kTileBytes);
+  const int code = (kBKernelDkdvFull << 12) | (kBRoleMma << 8);
+  uint32_t g = 0;        // steps whose S^T and dP^T are issued
+  uint32_t b_cnt = 0;    // steps whose dV and dK are issued
+  int acc_items = 0;     // items whose accumulators are complete (AccDone committed)
+  int items = 0;
+  bool ok = true;
+  bool pend = false, pend_first = false, pend_last = false;  // step g-1's dV, dK still to issue
+  uint32_t pend_slot = 0;
+  auto issue_b = [&]() -> bool {
+    if (!w.wait_warp(bar(kPFull), b_cnt & 1, code | kPFull)) return false;
+    if (pend_first && acc_items > 0 && !w.wait_warp(bar(L::kAccFree), (acc_items - 1) & 1, code | L::kAccFree))
+      return false;
+    tc_fence_after_sync();
+    const uint32_t qaddr = sbase + L::kRingOff + pend_slot * 2 * L::kTileBytes;
+    const uint64_t qb = mnmajor_desc<D>(qaddr), dob = mnmajor_desc<D>(qaddr + L::kTileBytes);
+    // dK first: the slot's Q, which the next S^T of that slot needs, is released first.
+#pragma unroll
+    for (int kk = 0; kk < kTile / 16; ++kk)
+      mma_bf16_ts_elect(t_dk, tY + 64 + kk * 8, qb + ((kk * 2048) >> 4), idesc_ts, (kk > 0 || !pend_first) ? 1u : 0u);
+    tc_commit_elect(bar(L::kRingEmpty + pend_slot));  // that step's Q is read
+#pragma unroll
+    for (int kk = 0; kk < kTile / 16; ++kk)
+      mma_bf16_ts_elect(t_dv, tY + kk * 8, dob + ((kk * 2048) >> 4), idesc_ts, (kk > 0 || !pend_first) ? 1u : 0u);
+    tc_commit_elect(bar(L::kRing2Empty + pend_slot));  // and its dO
+    if (pend_last) {
+      tc_commit_elect(bar(L::kAccDone));
+      ++acc_items;
+    }
+    ++b_cnt;
+    pend = false;
+    return true;
+  };
+  for (int i = blockIdx.x; ok && i < p.num_items; i += gridDim.x, ++items) {
+    const DkvItem it = dkv_item(p, i);
+    if (!w.wait_warp(bar(L::kFixFull), items & 1, code | L::kFixFull)) break;
+    tc_fence_after_sync();
+    for (int s = 0; s < it.steps; ++s, ++g) {
+      const uint32_t slot = g % L::kStages;
+      if (!w.wait_warp(bar(L::kRingFull + slot), (g / L::kStages) & 1, code | (L::kRingFull + slot)) ||
+          (g > 0 && !w.wait_warp(bar(kXFree), (g - 1) & 1, code | kXFree))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t qaddr = sbase + L::kRingOff + slot * 2 * L::kTileBytes;
+      const uint64_t q_desc = kmajor_desc<D>(qaddr), do_desc = kmajor_desc<D>(qaddr + L::kTileBytes);
+      // (dO of this slot is waited for below, before dP^T.)
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = kmajor_off<D>(kk);
+        mma_bf16_ss_elect(tX, k_desc + off, q_desc + off, idesc_ss, kk > 0 ? 1u : 0u);
+      }
+      tc_commit_elect(bar(kSFull));
+      if (pend && !issue_b()) {
+        ok = false;
+        break;
+      }
+      if (!w.wait_warp(bar(L::kRing2Full + slot), (g / L::kStages) & 1, code | (L::kRing2Full + slot))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = kmajor_off<D>(kk);
+        mma_bf16_ss_elect(tY, v_desc + off, do_desc + off, idesc_ss, kk > 0 ? 1u : 0u);
+      }
+      tc_commit_elect(bar(kDpFull));
+      if (s == it.steps - 1) tc_commit_elect(bar(L::kFixEmpty));  // K and V read by the item's last products
+      pend = true;
+      pend_slot = slot;
+      pend_first = (s == 0);
+      pend_last = (s == it.steps - 1);
+    }
+  }
+  if (ok && pend) issue_b();  // the last step's dV, dK
+}
+
+template <int D>
+__device__ __forceinline__ void dkvf_elem(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w,
+                                          int warp, int lane) {
+  using L = BwdSmem<D>;
+  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
+  constexpr int kSFull = L::kSFull, kDpFull = L::kSFull + 1;
+  constexpr int kPFull = L::kPFull, kXFree = L::kPFull + 1;
+  const int r = warp * 32 + lane;  // key row of the tile = TMEM lane
+  const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t tX = tmem + lane_bits, tY = tmem + lane_bits + 128;
+  const uint32_t t_dv = tmem + lane_bits + L::kColAcc0, t_dk = tmem + lane_bits + L::kColAcc1;
+  // Per-step query vectors, as in the half-tile kernel: copied a step ahead, then negated.
+  const uint32_t vec_saddr = sbase + L::kVecOff + warp * 4 * kTile * 4;
+  float* const vec_base = reinterpret_cast<float*>(__cvta_shared_to_generic(vec_saddr));
+  auto fetch_vectors = [&](int b, int hq, int m, uint32_t buf) {
+    const size_t bhq = (static_cast<size_t>(b) * p.Hq + hq) * p.N;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int c = lane + 32 * t, q = m * kTile + c;
+      const bool in = q < p.N;
+      const size_t idx = bhq + (in ? q : 0);
+      const uint32_t dst = vec_saddr + (buf * 2 * kTile + c) * 4;
+      cp_async_4(dst, p.lse + idx, in ? 4u : 0u);
+      cp_async_4(dst + kTile * 4, p.delta + idx, in ? 4u : 0u);
+    }
+    cp_async_commit();
+  };
+  const float c2 = p.scale_log2;
+  const uint64_t c2x2 = f32x2_pack(c2, c2);
+  const int code = (kBKernelDkdvFull << 12) | (kBRoleElem << 8);
+  uint32_t g = 0;
+  bool fetched = false;
+  int items = 0;
+  for (int i = blockIdx.x; i < p.num_items; i += gridDim.x, ++items) {
+    const DkvItem it = dkv_item(p, i);
+    const int key = it.n * kTile + r;
+    bool ok = true;
+    for (int s = 0; s < it.steps && ok; ++s, ++g) {
+      int hq, m;
+      dkv_step(p, it, s, hq, m);
+      const uint32_t buf = g & 1;
+      float* const s_lse = vec_base + buf * 2 * kTile;
+      float* const s_dlt = s_lse + kTile;
+      {
+        if (!fetched) fetch_vectors(it.b, hq, m, buf);
+        cp_async_wait_all();
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int c = lane + 32 * t;
+          s_lse[c] = -s_lse[c] * kLog2e;
+          s_dlt[c] = -s_dlt[c];
+        }
+        __syncwarp();
+        fetched = false;
+        if (s + 1 < it.steps) {
+          int hq2, m2;
+          dkv_step(p, it, s + 1, hq2, m2);
+          fetch_vectors(it.b, hq2, m2, buf ^ 1);
+          fetched = true;
+        } else if (i + static_cast<int>(gridDim.x) < p.num_items) {
+          const DkvItem nx = dkv_item(p, i + gridDim.x);
+          int hq2, m2;
+          dkv_step(p, nx, 0, hq2, m2);
+          fetch_vectors(nx.b, hq2, m2, buf ^ 1);
+          fetched = true;
+        }
+      }
+      // S^T of the step: load it, release X for the next step's product, mask.
+      if (!w.wait_warp(bar(kSFull), g & 1, code | kSFull)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      uint32_t sv[128];
+      tmem_load_128cols(tX, sv);
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kXFree));
+      if (block_is_partial(p, m, it.n)) {
+        // Query columns that see this key: lo_c <= c <= hi_c.
+        const int q0 = m * kTile;
+        const int hi_c =
+            (key < p.N) ? min(p.N - 1, p.mask_kind == kBMaskWindow ? key + p.window - 1 : p.N - 1) - q0 : -1;
+        const int lo_c = (p.mask_kind == kBMaskFull) ? 0 : key - q0;
+#pragma unroll
+        for (int c = 0; c < kTile; ++c)
+          if (c > hi_c || c < lo_c) sv[c] = 0xff800000u;  // -inf
+      }
+      // P^T = 2^(S c - lse log2 e), rounded to bf16 (query pairs per 32-bit word).
+      uint32_t pk[kTile / 2];
+#pragma unroll
+      for (int c = 0; c < kTile; c += 2) {
+        const float2 nl = *reinterpret_cast<const float2*>(s_lse + c);
+        float x0, x1;
+        f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), c2x2,
+                               f32x2_pack(nl.x, nl.y)),
+                     x0, x1);
+        pk[c >> 1] = bf16x2_rn(bexp2(x0), bexp2(x1));
+      }
+      // dS^T = P (dP - D) once dP^T is in Y, 32 queries at a time; P^T and dS^T go
+      // over Y only where dP^T has been read.
+      if (!w.wait_warp(bar(kDpFull), g & 1, code | kDpFull)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      uint32_t dk[kTile / 2];
+#pragma unroll
+      for (int chunk = 0; chunk < 4; ++chunk) {
+        uint32_t pv[32];
+        tmem_load_32cols(tY + chunk * 32, pv);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int c = chunk * 32 + e;
+          const float2 nd = *reinterpret_cast<const float2*>(s_dlt + c);
+          const uint32_t pw = pk[c >> 1];
+          float d0, d1;
+          f32x2_unpack(f32x2_mul(f32x2_pack(__uint_as_float(pw << 16), __uint_as_float(pw & 0xffff0000u)),
+                                 f32x2_add(f32x2_pack(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1])),
+                                           f32x2_pack(nd.x, nd.y))),
+                       d0, d1);
+          dk[c >> 1] = bf16x2_rn(d0, d1);
+        }
+        if (chunk == 1) tmem_store_32cols(tY, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));  // Y[0, 32) read
+      }
+      tmem_store_32cols(tY + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+      tmem_store_32cols(tY + 64, *reinterpret_cast<const uint32_t(*)[32]>(&dk[0]));
+      tmem_store_32cols(tY + 96, *reinterpret_cast<const uint32_t(*)[32]>(&dk[32]));
+      tmem_store_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kPFull));
+    }
+    if (!ok) break;
+    if (!w.wait_warp(bar(L::kAccDone), items & 1, code | L::kAccDone)) break;
+    tc_fence_after_sync();
+    const bool key_ok = key < p.N;
+    const size_t krow = (static_cast<size_t>(it.b) * p.Hkv + it.hkv) * p.N + (key_ok ? key : 0);
+    store_acc_row<D>(t_dv, 1.f, p.dv + krow * D, key_ok);
+    store_acc_row<D>(t_dk, p.scale, p.dk + krow * D, key_ok);
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(L::kAccFree));
+  }
+  cp_async_wait_all();
+  tmem_store_wait();
+}
+
 // Fused kernel, warps 6-9: after each dQ^T_h product, read it out of TMEM
 // (thread = TMEM lane = column c of dQ, 64 query values) and add it into the
 // fp32 accumulator: for each query, the warp's 32 lanes add 32 consecutive
@@ -961,6 +1402,10 @@ __global__ void __launch_bounds__(bwd_threads<KIND>(), 1) __maxnreg__(KIND == kB
       mbar_init(bar(L::kDqFree + h), 4);  // one arrival per dQ warp
     }
     mbar_init(bar(L::kDsFree), 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar(L::kRing2Full + s), 1);
+      mbar_init(bar(L::kRing2Empty + s), 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -976,17 +1421,21 @@ __global__ void __launch_bounds__(bwd_threads<KIND>(), 1) __maxnreg__(KIND == kB
   const BwdWaiter w{p.timeout_ns, abort_flag, p.err};
   if (warp < 4) {
     if constexpr (KIND == kBKernelDq) dq_elem<D>(p, sbase, tmem, w, warp, lane);
+    else if constexpr (KIND == kBKernelDqFull) dqf_elem<D>(p, sbase, tmem, w, warp, lane);
+    else if constexpr (KIND == kBKernelDkdvFull) dkvf_elem<D>(p, sbase, tmem, w, warp, lane);
     else dkv_elem<D, KIND == kBKernelFused>(p, sbase, tmem, w, warp, lane);
   } else if (warp >= kBwdDqWarp0) {
     if constexpr (KIND == kBKernelFused) dkv_dq<D>(p, sbase, tmem, w, warp, lane);
   } else if (warp == kBwdLoaderWarp) {
     if (lane == 0) {
-      if (KIND == kBKernelDq) dq_loader<D>(p, sbase, w);
-      else dkv_loader<D>(p, sbase, w);
+      if (KIND == kBKernelDq || KIND == kBKernelDqFull) dq_loader<D>(p, sbase, w);
+      else dkv_loader<D, KIND == kBKernelDkdvFull>(p, sbase, w);
     }
     __syncwarp();
   } else if (warp == kBwdMmaWarp) {
     if constexpr (KIND == kBKernelDq) dq_mma<D>(p, sbase, tmem, w);
+    else if constexpr (KIND == kBKernelDqFull) dqf_mma<D>(p, sbase, tmem, w);
+    else if constexpr (KIND == kBKernelDkdvFull) dkvf_mma<D>(p, sbase, tmem, w);
     else dkv_mma<D, KIND == kBKernelFused>(p, sbase, tmem, w);
     // Every MMA this warp issued must complete before TMEM is freed.
     tc_commit_elect(sbase + L::kBarOff + 8u * L::kFin);

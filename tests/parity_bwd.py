@@ -2,7 +2,9 @@
 
 Bound (derived from the arithmetic of the CUDA path): the kernels recompute P = exp(S - lse) in fp32, round P and
 dS = P (dP - D) to bf16 (relative error <= 2^-9 each, round to nearest) before
-the P^T dO, dS K and dS^T Q products, take D from the forward's bf16 output O
+the P^T dO, dS K and dS^T Q products (the full-tile kernels of the two-kernel
+path form dS from the bf16-rounded P: two roundings, <= 2^-8 relative, which
+the factor-of-two margin below covers), take D from the forward's bf16 output O
 (|D - D_exact| <= 2^-9 sum_c |dO_c O_c|), accumulate in fp32 and round each
 gradient to bf16 once (<= 2^-9 relative).  With a factor-of-two margin on
 each term, for every element

@@ -48,17 +48,18 @@ def test_deterministic_path_d128(cuda_ok, mask, window):
 
 
 def test_fused_and_deterministic_agree(cuda_ok):
-    """Both d = 128 paths on the same inputs: dk, dv bit for bit (the same key-tile code
-    forms them), dq close (the two paths form dS from S and from S^T, whose fp32 sums may
-    round differently, and add dQ's terms in different orders; each path meets the
-    oracle's bound in the tests above)."""
+    """Both d = 128 paths on the same inputs agree to the relative-L2 bar of the parity
+    tests. They differ only in rounding: the two-kernel path forms dS from the
+    bf16-rounded P (its full-tile kernels keep P as bf16 until dP arrives), the fused
+    path from fp32 P, and the paths add dQ's terms in different orders. Each path meets
+    the oracle's element bound in the tests above."""
     q, k, v = (t.cuda() for t in make_qkv(1, 4, 4, 1500, 128, 33))
     do = make_dout(1, 4, 1500, 128, 33).cuda()
     a = run_cuda_bwd(q, k, v, do, "causal")
     b = run_cuda_bwd(q, k, v, do, "causal", deterministic=True)
-    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
-    diff = (a[0].float() - b[0].float()).norm() / b[0].float().norm()
-    assert float(diff) < 2e-3, float(diff)
+    for x, y in zip(a, b):
+        diff = (x.float() - y.float()).norm() / y.float().norm()
+        assert float(diff) < 1e-2, float(diff)
 
 
 def test_multi_tile_and_scale(cuda_ok):
