@@ -1,8 +1,9 @@
 // Host side of the backward entry points declared in include/attn.h: argument
 // checks, TMA tensor maps and the launches on the caller's stream: D, then for
-// d = 128 the zeroed fp32 dQ accumulator, the fused key-tile kernel and the dQ
-// conversion; for d = 64 (or d = 128 with bwd_deterministic) the query-tile (dQ)
-// and key-tile (dK, dV) kernels.
+// d = 128 with Hq == Hkv the zeroed fp32 dQ accumulator, the fused key-tile
+// kernel and the dQ conversion; otherwise (d = 64, grouped heads, or
+// bwd_deterministic) the query-tile (dQ) and key-tile (dK, dV) kernels on whole
+// 128 x 128 tiles.
 #include "attn.h"
 
 #include <cuda.h>
@@ -79,9 +80,7 @@ int bwd_device_setup(BwdDevice& out) {
       void* addr = nullptr;
       if (cudaGetSymbolAddress(&addr, g_attn_bwd_error) != cudaSuccess) return ATTN_ERR_CUDA;
       info.err_word = static_cast<int*>(addr);
-      if (set_smem<64, kBKernelDq>() != cudaSuccess || set_smem<64, kBKernelDkdv>() != cudaSuccess ||
-          set_smem<128, kBKernelDq>() != cudaSuccess || set_smem<128, kBKernelDkdv>() != cudaSuccess ||
-          set_smem<128, kBKernelFused>() != cudaSuccess || set_smem<64, kBKernelDkdvFull>() != cudaSuccess ||
+      if (set_smem<128, kBKernelFused>() != cudaSuccess || set_smem<64, kBKernelDkdvFull>() != cudaSuccess ||
           set_smem<128, kBKernelDkdvFull>() != cudaSuccess || set_smem<64, kBKernelDqFull>() != cudaSuccess ||
           set_smem<128, kBKernelDqFull>() != cudaSuccess)
         return ATTN_ERR_CUDA;

@@ -10,24 +10,25 @@
 //   dQ = scale dS K,  dK = scale dS^T Q,
 // and grouped KV heads sum the gradients of the query heads that read them.
 //
-// Kernels, all on the caller's stream:
-//   attn_bwd_delta_kernel  D = rowsum(dO * O) in fp32 (the caller's workspace)
-//   the key-tile kernel    one 128-key K/V tile per work item, walking the
-//                          visible query tiles of every query head of its KV
-//                          group: S^T = K Q^T, dP^T = V dO^T, P^T and dS^T by
-//                          the elementwise warps, dV += P^T dO, dK += dS^T Q
-//                          (accumulated in TMEM over the item)
-// and, for dQ, one of two designs:
-//   d = 128: the key-tile kernel also forms dQ^T = K^T dS^T for each 64-query
-//            half (dS^T staged in shared memory), four more warps read it from
-//            TMEM and add it into an fp32 dQ accumulator in the workspace with
-//            coalesced global reductions, and attn_bwd_dq_convert_kernel
-//            scales and rounds the sums to bf16.  P and dS are formed once
-//            per (query, key) pair: five matmuls per pair.
-//   d = 64:  a query-tile kernel (one 128-row query tile per work item,
-//            walking its visible K/V tiles: S = Q K^T and dP = dO V^T
-//            recomputed, dS by the elementwise warps, dQ += dS K in TMEM),
-//            seven matmuls per pair and no atomics.
+// Kernels, all on the caller's stream, after attn_bwd_delta_kernel (D =
+// rowsum(dO * O) in fp32, in the caller's workspace).  A key-tile kernel takes
+// one 128-key K/V tile per work item and walks the visible query tiles of every
+// query head of its KV group: S^T = K Q^T, dP^T = V dO^T, P^T and dS^T by the
+// elementwise warps, dV += P^T dO and dK += dS^T Q accumulated in TMEM over the
+// item.  Two paths use it:
+//   fused (d = 128, Hq == Hkv): the key-tile kernel works in 64-query halves
+//            and also forms dQ^T = K^T dS^T for each half (dS^T staged in
+//            shared memory); four more warps read it from TMEM and add it into
+//            an fp32 dQ accumulator in the workspace with coalesced global
+//            reductions, and attn_bwd_dq_convert_kernel scales and rounds the
+//            sums to bf16.  P and dS are formed once per (query, key) pair:
+//            five matmuls per pair.
+//   two-kernel (d = 64, grouped heads, or on request): a query-tile kernel
+//            (one 128-row query tile per work item, walking its visible K/V
+//            tiles: S = Q K^T and dP = dO V^T recomputed, dS by the elementwise
+//            warps, dQ += dS K in TMEM), then the key-tile kernel for dK and
+//            dV; both on whole 128 x 128 tiles, seven matmuls per pair, no
+//            atomics.
 //
 // CTA organisation of the tcgen05 kernels (one CTA per SM, persistent):
 // warps 0-3 elementwise (thread = TMEM lane = one row of the work item's
@@ -300,7 +301,7 @@ __device__ __forceinline__ void store_acc_row(uint32_t tacc, float mul, __nv_bfl
   }
 }
 
-// ------------------------------------------------------------------ dQ kernel
+// ------------------------------------------------------------------ query-tile work items and loader
 struct DqItem {
   int b, hq, hkv, m, lo, hi;
 };
@@ -370,162 +371,7 @@ __device__ __forceinline__ void dq_loader(const BwdParams& p, uint32_t sbase, co
     w.drain(bar(L::kFixFull), (fix_issued - 1) & 1, (kBKernelDq << 12) | (kBRoleLoader << 8) | L::kFixFull);
 }
 
-template <int D>
-__device__ __forceinline__ void dq_mma(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w) {
-  using L = BwdSmem<D>;
-  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
-  constexpr uint32_t idesc_ss = idesc_bf16_f32(kTile, kHalf, false);  // 128 x 64 score halves
-  constexpr uint32_t idesc_ts = idesc_bf16_f32(kTile, D, true);
-  const uint32_t t_acc = tmem + L::kColAcc0;
-  const uint64_t q_desc = kmajor_desc<D>(sbase + L::kFixOff);
-  const uint64_t do_desc = kmajor_desc<D>(sbase + L::kFixOff + L::kTileBytes);
-  const int code = (kBKernelDq << 12) | (kBRoleMma << 8);
-  uint32_t n = 0;
-  uint32_t p_cnt0 = 0, p_cnt1 = 0;  // P / dS halves consumed, per half
-  int items = 0;
-  bool ok = true;
-  // dQ += dS_h K_h for half h of the key tile in ring slot `slot`.
-  auto issue_dq = [&](int h, uint32_t slot, bool first) -> bool {
-    if (!w.wait_warp(bar(L::kPFull + h), (h ? p_cnt1 : p_cnt0) & 1, code | (L::kPFull + h))) return false;
-    if (h) ++p_cnt1; else ++p_cnt0;
-    if (first && items > 0 && !w.wait_warp(bar(L::kAccFree), (items - 1) & 1, code | L::kAccFree)) return false;
-    tc_fence_after_sync();
-    const uint64_t kb = mnmajor_desc<D>(sbase + L::kRingOff + slot * 2 * L::kTileBytes) + ((h * kHalf * 128) >> 4);
-#pragma unroll
-    for (int kk = 0; kk < kHalf / 16; ++kk)
-      mma_bf16_ts_elect(t_acc, tmem + L::col_s(h) + kk * 8, kb + ((kk * 2048) >> 4), idesc_ts,
-                        (kk > 0 || !first) ? 1u : 0u);
-    return true;
-  };
-  for (int i = blockIdx.x; ok && i < p.num_items; i += gridDim.x, ++items) {
-    const DqItem it = dq_item(p, i);
-    if (!w.wait_warp(bar(L::kFixFull), items & 1, code | L::kFixFull)) break;
-    tc_fence_after_sync();
-    uint32_t prev_slot = 0;
-    bool first_dq = true;
-    for (int j = it.lo; j <= it.hi && ok; ++j, ++n) {
-      const uint32_t slot = n % L::kStages;
-      const uint32_t kaddr = sbase + L::kRingOff + slot * 2 * L::kTileBytes;
-      if (!w.wait_warp(bar(L::kRingFull + slot), (n / L::kStages) & 1, code | (L::kRingFull + slot))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after_sync();
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        // S_h = Q K_h^T and dP_h = dO V_h^T (keys 64h .. 64h+63 of the tile).
-        const uint64_t k_desc = kmajor_desc<D>(kaddr + h * kHalf * 128);
-        const uint64_t v_desc = kmajor_desc<D>(kaddr + L::kTileBytes + h * kHalf * 128);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = kmajor_off<D>(kk);
-          mma_bf16_ss_elect(tmem + L::col_s(h), q_desc + off, k_desc + off, idesc_ss, kk > 0 ? 1u : 0u);
-          mma_bf16_ss_elect(tmem + L::col_p(h), do_desc + off, v_desc + off, idesc_ss, kk > 0 ? 1u : 0u);
-        }
-        tc_commit_elect(bar(L::kSFull + h));
-        if (j == it.hi && h == 1) tc_commit_elect(bar(L::kFixEmpty));  // Q, dO read
-        // dQ for the half before this one: (j, 0) now, or (j - 1, 1) at h = 0.
-        if (h == 1 || j > it.lo) {
-          if (!issue_dq(1 - h, h == 1 ? slot : prev_slot, first_dq)) {
-            ok = false;
-            break;
-          }
-          first_dq = false;
-          if (h == 0) tc_commit_elect(bar(L::kRingEmpty + prev_slot));  // previous K, V tile done
-        }
-      }
-      prev_slot = slot;
-    }
-    if (!ok) break;
-    if (!issue_dq(1, prev_slot, first_dq)) break;  // the item's last half
-    tc_commit_elect(bar(L::kRingEmpty + prev_slot));
-    tc_commit_elect(bar(L::kAccDone));
-  }
-}
-
-template <int D>
-__device__ __forceinline__ void dq_elem(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w,
-                                        int warp, int lane) {
-  using L = BwdSmem<D>;
-  auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
-  const int r = warp * 32 + lane;  // row of the query tile = TMEM lane
-  const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t t_acc = tmem + lane_bits + L::kColAcc0;
-  const float c2 = p.scale_log2;
-  const int code = (kBKernelDq << 12) | (kBRoleElem << 8);
-  uint32_t s_cnt = 0;  // key tiles processed (each has both halves)
-  int items = 0;
-  for (int i = blockIdx.x; i < p.num_items; i += gridDim.x, ++items) {
-    const DqItem it = dq_item(p, i);
-    const int row = it.m * kTile + r;
-    const bool row_ok = row < p.N;
-    const size_t bhrow = (static_cast<size_t>(it.b) * p.Hq + it.hq) * p.N + (row_ok ? row : 0);
-    const float lse2 = row_ok ? p.lse[bhrow] * kLog2e : 0.f;
-    const float dlt = row_ok ? p.delta[bhrow] : 0.f;
-    const uint64_t c2x2 = f32x2_pack(c2, c2), nlse2x2 = f32x2_pack(-lse2, -lse2), ndlt2 = f32x2_pack(-dlt, -dlt);
-    bool ok = true;
-    for (int j = it.lo; j <= it.hi && ok; ++j, ++s_cnt) {
-      const bool partial = block_is_partial(p, it.m, j);
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        if (!w.wait_warp(bar(L::kSFull + h), s_cnt & 1, code | (L::kSFull + h))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after_sync();
-        // Visible key columns of this row in the half: lo_c <= c <= hi_c
-        // (applied on partial tiles, where masked scores become -inf).
-        const int j0 = j * kTile + h * kHalf;
-        const int hi_c = row_ok ? min(p.N - 1, p.mask_kind == kBMaskFull ? p.N - 1 : row) - j0 : -1;
-        const int lo_c = (p.mask_kind == kBMaskWindow) ? row - p.window + 1 - j0 : 0;
-        const uint32_t t_s = tmem + lane_bits + L::col_s(h), t_p = tmem + lane_bits + L::col_p(h);
-        uint32_t packed[2][16];
-#pragma unroll
-        for (int chunk = 0; chunk < 2; ++chunk) {
-          uint32_t sv[32], pv[32];
-          tmem_load_2x32cols(t_s + chunk * 32, t_p + chunk * 32, sv, pv);
-          if (partial) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int c = chunk * 32 + e;
-              if (c > hi_c || c < lo_c) sv[e] = 0xff800000u;  // -inf
-            }
-          }
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            // Column pairs on packed fp32 operations: x = s c - lse, p = 2^x,
-            // dS = p (dP - D).
-            float x0, x1, d0, d1;
-            f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2x2, nlse2x2),
-                         x0, x1);
-            const uint64_t pr2 = f32x2_pack(bexp2(x0), bexp2(x1));
-            f32x2_unpack(f32x2_mul(pr2, f32x2_add(f32x2_pack(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1])),
-                                                  ndlt2)),
-                         d0, d1);
-            packed[chunk][e >> 1] = bf16x2_rn(d0, d1);
-          }
-        }
-        // dS (bf16, 32 columns) over the first half of this half's S columns.
-        tmem_store_16cols(t_s, packed[0]);
-        tmem_store_16cols(t_s + 16, packed[1]);
-        tmem_store_wait();
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::kPFull + h));
-      }
-    }
-    if (!ok) break;
-    if (!w.wait_warp(bar(L::kAccDone), items & 1, code | L::kAccDone)) break;
-    tc_fence_after_sync();
-    store_acc_row<D>(t_acc, p.scale, p.dq + bhrow * D, row_ok);
-    tc_fence_before_sync();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar(L::kAccFree));
-  }
-  tmem_store_wait();
-}
-
-// ------------------------------------------------------------------ dK/dV kernel
+// ------------------------------------------------------------------ key-tile work items and loader; the fused kernel (64-query halves)
 struct DkvItem {
   int b, hkv, n, qlo, qhi, steps;  // steps = group * (qhi - qlo + 1)
 };
@@ -616,10 +462,10 @@ __device__ __forceinline__ void dkv_loader(const BwdParams& p, uint32_t sbase, c
   if (fix_issued > 0) w.drain(bar(L::kFixFull), (fix_issued - 1) & 1, code | L::kFixFull);
 }
 
-template <int D, bool kFused>
+template <int D>
 __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w) {
   using L = BwdSmem<D>;
-  static_assert(!kFused || D == 128, "the fused dQ^T product has M = d = 128");
+  static_assert(D == 128, "the fused dQ^T product has M = d = 128");
   auto bar = [&](int i) { return sbase + L::kBarOff + 8u * i; };
   constexpr uint32_t idesc_ss = idesc_bf16_f32(kTile, kHalf, false);  // 128 keys x 64 queries
   constexpr uint32_t idesc_ts = idesc_bf16_f32(kTile, D, true);
@@ -632,7 +478,7 @@ __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint
   const uint32_t t_dv = tmem + L::kColAcc0, t_dk = tmem + L::kColAcc1;
   const uint64_t k_desc = kmajor_desc<D>(sbase + L::kFixOff);
   const uint64_t v_desc = kmajor_desc<D>(sbase + L::kFixOff + L::kTileBytes);
-  const int code = ((kFused ? kBKernelFused : kBKernelDkdv) << 12) | (kBRoleMma << 8);
+  const int code = (kBKernelFused << 12) | (kBRoleMma << 8);
   uint32_t n = 0;
   uint32_t p_cnt0 = 0, p_cnt1 = 0;  // P / dS halves consumed, per half
   int items = 0;
@@ -643,18 +489,16 @@ __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint
     if (h) ++p_cnt1; else ++p_cnt0;
     if (first && items > 0 && !w.wait_warp(bar(L::kAccFree), (items - 1) & 1, code | L::kAccFree)) return false;
     tc_fence_after_sync();
-    if constexpr (kFused) {
-      // dQ^T_h over this tile's 128 keys, into the dP^T columns of half h.  It goes
-      // ahead of dV and dK so that the dQ warps read it out while those execute:
-      // the next S^T into these columns waits for that read.
+    // dQ^T_h over this tile's 128 keys, into the dP^T columns of half h.  It goes
+    // ahead of dV and dK so that the dQ warps read it out while those execute:
+    // the next S^T into these columns waits for that read.
 #pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk)
-        mma_bf16_ss_elect(tmem + L::col_p(h), kt_desc + ((kk * 2048) >> 4), ds_desc + ((kk * 2048) >> 4), idesc_dq,
-                          kk > 0 ? 1u : 0u);
-      tc_commit_elect(bar(L::kDqFull + h));
-      tc_commit_elect(bar(L::kDsFree));
-      ++dq_cnt[h];
-    }
+    for (int kk = 0; kk < kTile / 16; ++kk)
+      mma_bf16_ss_elect(tmem + L::col_p(h), kt_desc + ((kk * 2048) >> 4), ds_desc + ((kk * 2048) >> 4), idesc_dq,
+                        kk > 0 ? 1u : 0u);
+    tc_commit_elect(bar(L::kDqFull + h));
+    tc_commit_elect(bar(L::kDsFree));
+    ++dq_cnt[h];
     const uint32_t qaddr = sbase + L::kRingOff + slot * 2 * L::kTileBytes + h * kHalf * 128;
     const uint64_t qb = mnmajor_desc<D>(qaddr), dob = mnmajor_desc<D>(qaddr + L::kTileBytes);
 #pragma unroll
@@ -681,15 +525,13 @@ __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint
       tc_fence_after_sync();
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
-        if constexpr (kFused) {
-          // The dQ warps have read the previous dQ^T_h out of these columns.
-          if (dq_cnt[h] > 0 &&
-              !w.wait_warp(bar(L::kDqFree + h), (dq_cnt[h] - 1) & 1, code | (L::kDqFree + h))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after_sync();
+        // The dQ warps have read the previous dQ^T_h out of these columns.
+        if (dq_cnt[h] > 0 &&
+            !w.wait_warp(bar(L::kDqFree + h), (dq_cnt[h] - 1) & 1, code | (L::kDqFree + h))) {
+          ok = false;
+          break;
         }
+        tc_fence_after_sync();
         // S^T_h = K Q_h^T and dP^T_h = V dO_h^T (queries 64h .. 64h+63 of the tile).
         const uint64_t q_desc = kmajor_desc<D>(qaddr + h * kHalf * 128);
         const uint64_t do_desc = kmajor_desc<D>(qaddr + L::kTileBytes + h * kHalf * 128);
@@ -700,7 +542,6 @@ __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint
           mma_bf16_ss_elect(tmem + L::col_p(h), v_desc + off, do_desc + off, idesc_ss, kk > 0 ? 1u : 0u);
         }
         tc_commit_elect(bar(L::kSFull + h));
-        if (!kFused && s == it.steps - 1 && h == 1) tc_commit_elect(bar(L::kFixEmpty));  // K, V read
         if (h == 1 || s > 0) {
           if (!issue_dkv(1 - h, h == 1 ? slot : prev_slot, first)) {
             ok = false;
@@ -714,13 +555,13 @@ __device__ __forceinline__ void dkv_mma(const BwdParams& p, uint32_t sbase, uint
     }
     if (!ok) break;
     if (!issue_dkv(1, prev_slot, first)) break;  // the item's last half
-    if (kFused) tc_commit_elect(bar(L::kFixEmpty));  // K (read by the dQ^T products too), V
+    tc_commit_elect(bar(L::kFixEmpty));  // K (read by the dQ^T products too), V
     tc_commit_elect(bar(L::kRingEmpty + prev_slot));
     tc_commit_elect(bar(L::kAccDone));
   }
 }
 
-template <int D, bool kFused>
+template <int D>
 __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uint32_t tmem, const BwdWaiter& w,
                                          int warp, int lane) {
   using L = BwdSmem<D>;
@@ -748,7 +589,7 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
   };
   const float c2 = p.scale_log2;
   const uint64_t c2x2 = f32x2_pack(c2, c2);
-  const int code = ((kFused ? kBKernelFused : kBKernelDkdv) << 12) | (kBRoleElem << 8);
+  const int code = (kBKernelFused << 12) | (kBRoleElem << 8);
   uint32_t s_cnt = 0;
   uint32_t ds_cnt = 0;  // fused kernel: dS^T halves staged in shared memory
   bool fetched = false;  // the next step's vectors are already on their way
@@ -795,14 +636,12 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
           ok = false;
           break;
         }
-        if constexpr (kFused) {
-          // The staged dS^T is rewritten below: the previous dQ^T product must have read it.
-          if (ds_cnt > 0 && !w.wait_warp(bar(L::kDsFree), (ds_cnt - 1) & 1, code | L::kDsFree)) {
-            ok = false;
-            break;
-          }
-          ++ds_cnt;
+        // The staged dS^T is rewritten below: the previous dQ^T product must have read it.
+        if (ds_cnt > 0 && !w.wait_warp(bar(L::kDsFree), (ds_cnt - 1) & 1, code | L::kDsFree)) {
+          ok = false;
+          break;
         }
+        ++ds_cnt;
         tc_fence_after_sync();
         // Query columns of this half that see the key: lo_c <= c <= hi_c
         // (applied on partial tiles, where masked scores become -inf).
@@ -844,17 +683,15 @@ __device__ __forceinline__ void dkv_elem(const BwdParams& p, uint32_t sbase, uin
             dk[chunk][e >> 1] = bf16x2_rn(d0, d1);
           }
         }
-        if constexpr (kFused) {
-          // Stage dS^T for dQ^T = K^T dS^T: this key's row of 64 queries is 128 B
-          // (eight 16-byte chunks, chunk c stored at c ^ (row & 7): the 128-byte
-          // swizzle of an MN-major operand).
-          const uint32_t row_addr = sbase + L::kDsOff + r * 128;
+        // Stage dS^T for dQ^T = K^T dS^T: this key's row of 64 queries is 128 B
+        // (eight 16-byte chunks, chunk c stored at c ^ (row & 7): the 128-byte
+        // swizzle of an MN-major operand).
+        const uint32_t row_addr = sbase + L::kDsOff + r * 128;
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            st_shared_v4(row_addr + ((c ^ (r & 7)) << 4), dk[c >> 2][(c & 3) * 4], dk[c >> 2][(c & 3) * 4 + 1],
-                         dk[c >> 2][(c & 3) * 4 + 2], dk[c >> 2][(c & 3) * 4 + 3]);
-          fence_proxy_async_smem();
-        }
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(row_addr + ((c ^ (r & 7)) << 4), dk[c >> 2][(c & 3) * 4], dk[c >> 2][(c & 3) * 4 + 1],
+                       dk[c >> 2][(c & 3) * 4 + 2], dk[c >> 2][(c & 3) * 4 + 3]);
+        fence_proxy_async_smem();
         // P^T and dS^T (bf16, 32 columns each) over this half's S^T columns.
         tmem_store_16cols(t_s, pk[0]);
         tmem_store_16cols(t_s + 16, pk[1]);
@@ -1420,23 +1257,21 @@ __global__ void __launch_bounds__(bwd_threads<KIND>(), 1) __maxnreg__(KIND == kB
   const uint32_t tmem = *tmem_slot;
   const BwdWaiter w{p.timeout_ns, abort_flag, p.err};
   if (warp < 4) {
-    if constexpr (KIND == kBKernelDq) dq_elem<D>(p, sbase, tmem, w, warp, lane);
-    else if constexpr (KIND == kBKernelDqFull) dqf_elem<D>(p, sbase, tmem, w, warp, lane);
+    if constexpr (KIND == kBKernelDqFull) dqf_elem<D>(p, sbase, tmem, w, warp, lane);
     else if constexpr (KIND == kBKernelDkdvFull) dkvf_elem<D>(p, sbase, tmem, w, warp, lane);
-    else dkv_elem<D, KIND == kBKernelFused>(p, sbase, tmem, w, warp, lane);
+    else dkv_elem<D>(p, sbase, tmem, w, warp, lane);
   } else if (warp >= kBwdDqWarp0) {
     if constexpr (KIND == kBKernelFused) dkv_dq<D>(p, sbase, tmem, w, warp, lane);
   } else if (warp == kBwdLoaderWarp) {
     if (lane == 0) {
-      if (KIND == kBKernelDq || KIND == kBKernelDqFull) dq_loader<D>(p, sbase, w);
+      if (KIND == kBKernelDqFull) dq_loader<D>(p, sbase, w);
       else dkv_loader<D, KIND == kBKernelDkdvFull>(p, sbase, w);
     }
     __syncwarp();
   } else if (warp == kBwdMmaWarp) {
-    if constexpr (KIND == kBKernelDq) dq_mma<D>(p, sbase, tmem, w);
-    else if constexpr (KIND == kBKernelDqFull) dqf_mma<D>(p, sbase, tmem, w);
+    if constexpr (KIND == kBKernelDqFull) dqf_mma<D>(p, sbase, tmem, w);
     else if constexpr (KIND == kBKernelDkdvFull) dkvf_mma<D>(p, sbase, tmem, w);
-    else dkv_mma<D, KIND == kBKernelFused>(p, sbase, tmem, w);
+    else dkv_mma<D>(p, sbase, tmem, w);
     // Every MMA this warp issued must complete before TMEM is freed.
     tc_commit_elect(sbase + L::kBarOff + 8u * L::kFin);
     w.drain(sbase + L::kBarOff + 8u * L::kFin, 0, (KIND << 12) | (kBRoleMma << 8) | L::kFin);
